@@ -1,0 +1,329 @@
+// kvq_abi.cu - the extern "C" entry points of libkvq.so (host code only).
+//
+// Validation happens here, before any launch; the launchers in kvq_append.cu,
+// kvq_decode.cu and kvq_dequant.cu only see consistent arguments.
+#include <cuda_runtime.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "kvq_internal.h"
+
+using namespace kvq;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+const char *type_name(int t) {
+  static const char *names[KVQ_TYPE_COUNT] = {
+      "bf16", "q2_0", "q3_0", "q4_0", "q5_0", "q6_0", "q8_0", "q4_1", "kvarn2", "kvarn3",
+      "kvarn4", "kvarn5", "kvarn6", "kvarn8", "q2_1", "q3_1", "q5_1", "q6_1"};
+  return (t >= 0 && t < KVQ_TYPE_COUNT) ? names[t] : "?";
+}
+
+int check_params(const kvq_params *p) {
+  if (!p) return KVQ_E_INVAL;
+  if (p->n_layers < 1 || p->n_seqs < 1 || p->n_kv_heads < 1 || p->max_ctx < 1 || p->tail < 0)
+    return KVQ_E_INVAL;
+  if (p->head_dim != D || p->group != GROUP || p->page_tokens != GROUP) return KVQ_E_UNSUPPORTED;
+  if (p->sinkhorn_iters < 1 || p->sinkhorn_iters > 64) return KVQ_E_INVAL;
+  TypeInfo tk = type_info(p->type_k), tv = type_info(p->type_v);
+  if (tk.fam < 0 || tv.fam < 0) return KVQ_E_UNSUPPORTED;
+  if ((tk.fam == FAM_BF16) != (tv.fam == FAM_BF16)) return KVQ_E_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+// Fills the derived geometry of a cache; returns the device bytes it needs.
+size_t plan(kvq_cache *c) {
+  const kvq_params &p = c->p;
+  TypeInfo tk = type_info(p.type_k), tv = type_info(p.type_v);
+  c->fam_k = tk.fam;
+  c->bits_k = tk.bits;
+  c->fam_v = tv.fam;
+  c->bits_v = tv.bits;
+  c->lk = sub_layout(tk.fam, tk.bits);
+  c->lv = sub_layout(tv.fam, tv.bits);
+  const bool bf16 = tk.fam == FAM_BF16;
+  c->max_pages = bf16 ? 0 : (p.max_ctx + GROUP - 1) / GROUP;
+  c->page_bytes = (int64_t)p.n_kv_heads * (c->lk.bytes + c->lv.bytes);
+  const bool any_kvarn = tk.fam == FAM_KVARN || tv.fam == FAM_KVARN;
+  c->ring_cap = bf16 ? p.max_ctx : (int64_t)p.tail + (any_kvarn ? GROUP : 0);
+  c->layer_pages_bytes = align_up((size_t)p.n_seqs * c->max_pages * c->page_bytes);
+  c->layer_ring_bytes = align_up((size_t)p.n_seqs * p.n_kv_heads * 2 * c->ring_cap * 2 * D);
+  size_t off = 0;
+  c->off_pages = off;
+  off += c->layer_pages_bytes * p.n_layers;
+  c->off_ring = off;
+  off += c->layer_ring_bytes * p.n_layers;
+  c->off_ptab = off;
+  off += align_up(sizeof(int32_t) * std::max<int64_t>(1, (int64_t)p.n_seqs * c->max_pages));
+  c->off_tickets = off;
+  off += align_up(sizeof(uint32_t) * (size_t)p.n_seqs * p.n_kv_heads);
+  c->off_status = off;
+  off += kAlign;
+  c->total = off;
+  return off;
+}
+
+}  // namespace
+
+namespace kvq {
+LayerView layer_view(const kvq_cache *c, int layer) {
+  LayerView L;
+  L.pages = c->base + c->off_pages + c->layer_pages_bytes * layer;
+  L.ring = c->base + c->off_ring + c->layer_ring_bytes * layer;
+  L.ptab = reinterpret_cast<const int32_t *>(c->base + c->off_ptab);
+  L.status = reinterpret_cast<int32_t *>(c->base + c->off_status);
+  L.max_pages = c->max_pages;
+  L.page_bytes = c->page_bytes;
+  L.ring_cap = c->ring_cap;
+  L.hkv = c->p.n_kv_heads;
+  L.sub_k = c->lk.bytes;
+  L.sub_v = c->lv.bytes;
+  L.type_k = c->p.type_k;
+  L.type_v = c->p.type_v;
+  return L;
+}
+}  // namespace kvq
+
+extern "C" {
+
+void kvq_default_params(kvq_params *p) {
+  if (!p) return;
+  memset(p, 0, sizeof *p);
+  p->n_layers = 1;
+  p->n_seqs = 1;
+  p->n_kv_heads = 8;
+  p->head_dim = D;
+  p->max_ctx = 65536;
+  p->type_k = KVQ_KVARN4;
+  p->type_v = KVQ_KVARN4;
+  p->tail = 1024;
+  p->group = GROUP;
+  p->sinkhorn_iters = 8;
+  p->page_tokens = GROUP;
+}
+
+int kvq_cache_bytes(const kvq_params *p, size_t *bytes) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (!bytes) return KVQ_E_INVAL;
+  kvq_cache tmp;
+  tmp.p = *p;
+  *bytes = plan(&tmp);
+  return KVQ_OK;
+}
+
+int kvq_payload_bytes(int32_t type, int32_t raw_bits, int64_t n_layers, int64_t n_kv_heads,
+                      int64_t n, int64_t tail, double *bytes) {
+  TypeInfo ti = type_info(type);
+  if (ti.fam < 0 || !bytes || n < 0 || tail < 0 || n_layers < 0 || n_kv_heads < 0 || raw_bits < 0)
+    return KVQ_E_INVAL;
+  int64_t keep = ti.fam == FAM_BF16 ? n : std::min(n, tail);
+  int64_t Q = n - keep;
+  double per = (double)keep * D * 2.0;
+  if (raw_bits > 0)
+    per += (double)Q * D * raw_bits / 8.0;
+  else if (Q > 0) {
+    per += (double)Q * token_bytes(ti.fam, ti.bits);
+    if (ti.fam == FAM_KVARN) per += (double)((Q + GROUP - 1) / GROUP) * 2.0 * D;
+  }
+  *bytes = per * 2.0 * (double)n_layers * (double)n_kv_heads;
+  return KVQ_OK;
+}
+
+int kvq_cache_create(const kvq_params *p, void *dev_buf, size_t bytes, kvq_cache **out) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (!dev_buf || !out) return KVQ_E_INVAL;
+  if (!aligned16(dev_buf)) return KVQ_E_ALIGN;
+  kvq_cache *c = new (std::nothrow) kvq_cache;
+  if (!c) return KVQ_E_INVAL;
+  c->p = *p;
+  size_t need = plan(c);
+  if (bytes < need) {
+    delete c;
+    return KVQ_E_SIZE;
+  }
+  c->base = static_cast<uint8_t *>(dev_buf);
+  c->bytes = bytes;
+  c->len.assign((size_t)p->n_layers * p->n_seqs, 0);
+  if (cudaGetDevice(&c->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+    delete c;
+    return KVQ_E_CUDA;
+  }
+  // static page table: sequence s, logical page j -> physical page s * max_pages + j
+  if (c->max_pages > 0) {
+    std::vector<int32_t> ptab((size_t)p->n_seqs * c->max_pages);
+    for (size_t i = 0; i < ptab.size(); ++i) ptab[i] = (int32_t)i;
+    if (cudaMemcpy(c->base + c->off_ptab, ptab.data(), ptab.size() * sizeof(int32_t),
+                   cudaMemcpyHostToDevice) != cudaSuccess) {
+      delete c;
+      return KVQ_E_CUDA;
+    }
+  }
+  if (cudaMemset(c->base + c->off_tickets, 0, c->total - c->off_tickets) != cudaSuccess) {
+    delete c;
+    return KVQ_E_CUDA;
+  }
+  *out = c;
+  return KVQ_OK;
+}
+
+void kvq_cache_destroy(kvq_cache *c) { delete c; }
+
+int kvq_append(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,
+               const int32_t *n_new, const void *k_bf16, const void *v_bf16, kvq_stream_t stream) {
+  if (!c || layer < 0 || layer >= c->p.n_layers || n_seqs < 0) return KVQ_E_INVAL;
+  if (n_seqs > 0 && (!seq_ids || !n_new)) return KVQ_E_INVAL;
+  std::vector<char> seen(c->p.n_seqs, 0);
+  std::vector<AppendSeq> seqs;
+  int64_t rows = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    int s = seq_ids[i];
+    if (s < 0 || s >= c->p.n_seqs || seen[s] || n_new[i] < 0) return KVQ_E_INVAL;
+    seen[s] = 1;
+    int64_t n0 = c->len[(size_t)layer * c->p.n_seqs + s];
+    if (n0 + n_new[i] > c->p.max_ctx) return KVQ_E_CAPACITY;
+    if (n_new[i] > 0) seqs.push_back({s, n_new[i], n0, rows});
+    rows += n_new[i];
+  }
+  if (rows == 0) return KVQ_OK;
+  if (!k_bf16 || !v_bf16) return KVQ_E_INVAL;
+  if (!aligned16(k_bf16) || !aligned16(v_bf16)) return KVQ_E_ALIGN;
+  int rc = launch_append(c, layer, seqs, k_bf16, v_bf16, reinterpret_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  for (const AppendSeq &a : seqs) c->len[(size_t)layer * c->p.n_seqs + a.seq] = a.n0 + a.n_new;
+  return KVQ_OK;
+}
+
+int kvq_workspace_bytes(const kvq_cache *c, int32_t n_seqs, int32_t n_q_heads, size_t *bytes) {
+  if (!c || !bytes || n_seqs < 0 || n_q_heads < 1) return KVQ_E_INVAL;
+  if (n_q_heads % c->p.n_kv_heads) return KVQ_E_INVAL;
+  if (n_q_heads / c->p.n_kv_heads > MAX_G) return KVQ_E_UNSUPPORTED;
+  *bytes = decode_workspace_bytes(c, n_seqs, n_q_heads);
+  return KVQ_OK;
+}
+
+int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,
+                    int32_t n_q_heads, const float *q, float softmax_scale, float *out, void *workspace,
+                    size_t ws_bytes, kvq_stream_t stream) {
+  if (!c || layer < 0 || layer >= c->p.n_layers || n_seqs < 0) return KVQ_E_INVAL;
+  if (n_seqs == 0) return KVQ_OK;
+  if (!seq_ids || !q || !out || !workspace || n_q_heads < 1) return KVQ_E_INVAL;
+  if (n_q_heads % c->p.n_kv_heads) return KVQ_E_INVAL;
+  if (n_q_heads / c->p.n_kv_heads > MAX_G) return KVQ_E_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_E_ALIGN;
+  if (ws_bytes < decode_workspace_bytes(c, n_seqs, n_q_heads)) return KVQ_E_SIZE;
+  std::vector<char> seen(c->p.n_seqs, 0);
+  std::vector<DecodeSeq> seqs;
+  for (int i = 0; i < n_seqs; ++i) {
+    int s = seq_ids[i];
+    if (s < 0 || s >= c->p.n_seqs || seen[s]) return KVQ_E_INVAL;
+    seen[s] = 1;
+    int64_t n = c->len[(size_t)layer * c->p.n_seqs + s];
+    seqs.push_back({s, i, n, quantized_len(c, n)});
+  }
+  float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
+  return launch_decode(c, layer, seqs, n_q_heads, q, scale, out, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int kvq_dequant(kvq_cache *c, int32_t layer, int32_t seq, int32_t which, int64_t t0, int64_t t1,
+                int32_t basis, float *out, kvq_stream_t stream) {
+  if (!c || layer < 0 || layer >= c->p.n_layers || seq < 0 || seq >= c->p.n_seqs) return KVQ_E_INVAL;
+  if (which < 0 || which > 1 || basis < 0 || basis > 1) return KVQ_E_INVAL;
+  int64_t n = c->len[(size_t)layer * c->p.n_seqs + seq];
+  if (t0 < 0 || t1 < t0 || t1 > n) return KVQ_E_INVAL;
+  if (t1 == t0) return KVQ_OK;
+  if (!out) return KVQ_E_INVAL;
+  if (!aligned16(out)) return KVQ_E_ALIGN;
+  return launch_dequant(c, layer, seq, which, t0, t1, basis, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int kvq_seq_len(const kvq_cache *c, int32_t layer, int32_t seq, int64_t *len) {
+  if (!c || !len || layer < 0 || layer >= c->p.n_layers || seq < 0 || seq >= c->p.n_seqs)
+    return KVQ_E_INVAL;
+  *len = c->len[(size_t)layer * c->p.n_seqs + seq];
+  return KVQ_OK;
+}
+
+int kvq_seq_reset(kvq_cache *c, int32_t seq) {
+  if (!c || seq < 0 || seq >= c->p.n_seqs) return KVQ_E_INVAL;
+  for (int l = 0; l < c->p.n_layers; ++l) c->len[(size_t)l * c->p.n_seqs + seq] = 0;
+  return KVQ_OK;
+}
+
+int kvq_locate(const kvq_cache *c, int32_t kind, int32_t layer, int32_t seq, int64_t page, int32_t head,
+               int32_t which, int64_t token, size_t *offset, size_t *bytes) {
+  if (!c || !offset || !bytes || layer < 0 || layer >= c->p.n_layers || seq < 0 || seq >= c->p.n_seqs ||
+      head < 0 || head >= c->p.n_kv_heads || which < 0 || which > 1)
+    return KVQ_E_INVAL;
+  if (kind == 0) {
+    if (page < 0 || page >= c->max_pages) return KVQ_E_INVAL;
+    int64_t phys = (int64_t)seq * c->max_pages + page;
+    *offset = c->off_pages + c->layer_pages_bytes * layer + phys * c->page_bytes +
+              (size_t)head * (c->lk.bytes + c->lv.bytes) + (which ? c->lk.bytes : 0);
+    *bytes = which ? c->lv.bytes : c->lk.bytes;
+    return KVQ_OK;
+  }
+  if (kind == 1) {
+    if (c->ring_cap == 0 || token < 0) return KVQ_E_INVAL;
+    *offset = c->off_ring + c->layer_ring_bytes * layer +
+              ((((size_t)seq * c->p.n_kv_heads + head) * 2 + which) * c->ring_cap + token % c->ring_cap) *
+                  (2 * D);
+    *bytes = 2 * D;
+    return KVQ_OK;
+  }
+  return KVQ_E_INVAL;
+}
+
+int kvq_get_status(kvq_cache *c, kvq_stream_t stream) {
+  if (!c) return KVQ_E_INVAL;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return KVQ_E_CUDA;
+  int32_t st = 0;
+  if (cudaMemcpy(&st, c->base + c->off_status, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KVQ_E_CUDA;
+  if (st != 0) {
+    cudaMemset(c->base + c->off_status, 0, sizeof st);
+    return KVQ_E_DEVICE;
+  }
+  return KVQ_OK;
+}
+
+const char *kvq_describe(kvq_cache *c) {
+  if (!c) return "";
+  char buf[512];
+  snprintf(buf, sizeof buf,
+           "kvq cache: K %s, V %s, tail %d (BF16), %d layers x %d seqs x %d KV heads x %d, max_ctx %lld, "
+           "sinkhorn_iters %d, %zu bytes (pages %zu/layer, ring %zu/layer)",
+           type_name(c->p.type_k), type_name(c->p.type_v), c->p.tail, c->p.n_layers, c->p.n_seqs,
+           c->p.n_kv_heads, c->p.head_dim, (long long)c->p.max_ctx, c->p.sinkhorn_iters, c->total,
+           c->layer_pages_bytes, c->layer_ring_bytes);
+  c->desc = buf;
+  return c->desc.c_str();
+}
+
+const char *kvq_strerror(int code) {
+  switch (code) {
+    case KVQ_OK: return "ok";
+    case KVQ_E_INVAL: return "invalid argument";
+    case KVQ_E_UNSUPPORTED: return "unsupported geometry or type";
+    case KVQ_E_CAPACITY: return "sequence capacity (max_ctx) exceeded";
+    case KVQ_E_ALIGN: return "device pointer not 16-byte aligned";
+    case KVQ_E_CUDA: return "CUDA error";
+    case KVQ_E_DEVICE: return "device status word reports an error";
+    case KVQ_E_SIZE: return "caller buffer too small";
+    default: return "unknown error";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,488 @@
+// kvq_append.cu - append path: tail ring write, spill quantization (qb_0, qb_1, kvarn).
+//
+// Compiled with -fmad=false and written with explicit __f*_rn intrinsics: every fp32
+// operation that decides a code or a scale rounds once, in the order written, so the
+// codes and fp16 scales match the CPU oracle bit for bit.
+//
+// Steps (pages: "KV Cache Precision Tail" and "KVarN" sections of the BeeLLama.cpp v0.4.0
+// page; "How WHT and Sinkhorn save quality at 4-bit" of the Bonsai-Ternary-27B page):
+//  1. tokens that leave the newest-`tail` window are quantized; for kvarn every 256-token
+//     group touched by the append is rebuilt from its BF16 rows (ring or new input):
+//     Walsh-Hadamard rotation -> Sinkhorn balancing -> symmetric block quantization;
+//  2. the new tokens that stay 16-bit are copied into the BF16 ring.
+// Step 1 reads ring rows that step 2 may overwrite, so step 2 is launched after it.
+#include <cuda_runtime.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int MAXS = 64;  // sequences per launch (kernel parameter space)
+
+struct SeqWork {
+  int32_t seq;
+  int32_t pad;
+  int64_t n0, n1;    // sequence length before / after the append
+  int64_t in_off;    // first input row of this sequence
+  int64_t a, b;      // kernel-specific range
+  int64_t item0;     // first work item of this sequence
+};
+
+struct Work {
+  int32_t n;
+  int32_t which;
+  int64_t total;
+  SeqWork s[MAXS];
+};
+
+__device__ __forceinline__ int find_seq(const Work &W, int64_t item) {
+  int si = 0;
+  while (si + 1 < W.n && W.s[si + 1].item0 <= item) ++si;
+  return si;
+}
+
+__device__ __forceinline__ const __nv_bfloat16 *src_row(const LayerView &L, const SeqWork &s, int head,
+                                                        int which, int64_t p, const __nv_bfloat16 *in) {
+  if (p < s.n0) return ring_row(L, s.seq, head, which, p);
+  return in + ((s.in_off + (p - s.n0)) * L.hkv + head) * D;
+}
+
+__device__ __forceinline__ void load4(const __nv_bfloat16 *row, int lane, float (&x)[4]) {
+  uint2 raw = *reinterpret_cast<const uint2 *>(row + 4 * lane);
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
+  x[0] = __low2float(a);
+  x[1] = __high2float(a);
+  x[2] = __low2float(b);
+  x[3] = __high2float(b);
+}
+
+// ---- packing -------------------------------------------------------------------------
+
+// K plane of width W: the warp's lane holds channels 4*jj..4*jj+3 of block blk (jj = lane&7).
+template <int W>
+__device__ __forceinline__ void pack_k_plane(const uint32_t (&v)[4], uint8_t *plane, int blk, int jj) {
+  constexpr int F = 8 / W;
+  constexpr uint32_t MASK = (1u << W) - 1u;
+  const int m = jj / F, s = jj % F;
+  uint32_t word = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) word |= (v[k] & MASK) << (8 * k + s * W);
+#pragma unroll
+  for (int o = 1; o < F; o <<= 1) word |= __shfl_xor_sync(FULL, word, o);
+  if (s == 0) *reinterpret_cast<uint32_t *>(plane + 16 * m + 4 * blk) = word;
+}
+
+// V plane of width W for quad token k: the lane holds channels 4*j8..4*j8+3 of block blk.
+template <int W>
+__device__ __forceinline__ void pack_v_plane(const uint32_t (&v)[4], uint8_t *plane, int blk, int j8, int k) {
+  constexpr uint32_t MASK = (1u << W) - 1u;
+  uint8_t *base = plane + 16 * W * blk + k;
+  if constexpr (W == 8) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) base[4 * (4 * j8 + i)] = (uint8_t)(v[i] & MASK);
+  } else if constexpr (W == 4) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      base[4 * (2 * j8 + h)] = (uint8_t)((v[2 * h] & MASK) | ((v[2 * h + 1] & MASK) << 4));
+  } else if constexpr (W == 2) {
+    base[4 * j8] = (uint8_t)((v[0] & MASK) | ((v[1] & MASK) << 2) | ((v[2] & MASK) << 4) | ((v[3] & MASK) << 6));
+  } else {  // W == 1: two lanes share one byte
+    uint32_t nib = (v[0] & 1u) | ((v[1] & 1u) << 1) | ((v[2] & 1u) << 2) | ((v[3] & 1u) << 3);
+    nib <<= 4 * (j8 & 1);
+    nib |= __shfl_xor_sync(FULL, nib, 1);
+    if ((j8 & 1) == 0) base[4 * (j8 >> 1)] = (uint8_t)nib;
+  }
+}
+
+template <int BITS, int WHICH>
+__device__ __forceinline__ void pack_codes(const int (&code)[4], uint8_t *sub, int tip, int lane) {
+  constexpr int WL = plane_lo(BITS), WH = plane_hi(BITS);
+  uint32_t lo[4], hi[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    uint32_t f = (uint32_t)code[e] & ((1u << BITS) - 1u);
+    lo[e] = f & ((1u << WL) - 1u);
+    hi[e] = f >> WL;
+  }
+  const int blk = lane >> 3, j8 = lane & 7;
+  if constexpr (WHICH == 0) {
+    uint8_t *tok = sub + tip * 16 * BITS;
+    pack_k_plane<WL>(lo, tok, blk, j8);
+    if constexpr (WH > 0) pack_k_plane<WH>(hi, tok + 16 * WL, blk, j8);
+  } else {
+    uint8_t *quad = sub + (tip >> 2) * 64 * BITS;
+    pack_v_plane<WL>(lo, quad, blk, j8, tip & 3);
+    if constexpr (WH > 0) pack_v_plane<WH>(hi, quad + 64 * WL, blk, j8, tip & 3);
+  }
+}
+
+// ---- block quantizers (one token-head per warp; lane holds channels 4*lane..+3) ------
+
+template <int BITS, int WHICH>
+__device__ __forceinline__ void quant_sym(const float (&y)[4], uint8_t *sub, const SubLayout &lay, int tip,
+                                          int lane) {
+  constexpr int QMAX = (1 << (BITS - 1)) - 1, QMIN = -(1 << (BITS - 1));
+  float a = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+  a = fmaxf(a, __shfl_xor_sync(FULL, a, 4));
+  a = fmaxf(a, __shfl_xor_sync(FULL, a, 2));
+  a = fmaxf(a, __shfl_xor_sync(FULL, a, 1));
+  const __half dh = sat_half(__fdiv_rn(a, (float)QMAX));
+  const float df = __half2float(dh);
+  int code[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    int q = 0;
+    if (df != 0.0f) {
+      float r = rintf(__fdiv_rn(y[e], df));
+      r = fminf(fmaxf(r, (float)QMIN), (float)QMAX);
+      q = (int)r;
+    }
+    code[e] = q;
+  }
+  pack_codes<BITS, WHICH>(code, sub, tip, lane);
+  if ((lane & 7) == 0) reinterpret_cast<__half *>(sub + lay.d)[tip * 4 + (lane >> 3)] = dh;
+}
+
+template <int BITS, int WHICH>
+__device__ __forceinline__ void quant_asym(const float (&x)[4], uint8_t *sub, const SubLayout &lay, int tip,
+                                           int lane) {
+  constexpr int QMAX = (1 << BITS) - 1;
+  float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+  float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+#pragma unroll
+  for (int o = 4; o >= 1; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+  }
+  const __half dh = sat_half(__fdiv_rn(__fsub_rn(mx, mn), (float)QMAX));
+  const __half mh = sat_half(mn);
+  const float df = __half2float(dh), mf = __half2float(mh);
+  int code[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    int q = 0;
+    if (df != 0.0f) {
+      float r = rintf(__fdiv_rn(__fsub_rn(x[e], mf), df));
+      r = fminf(fmaxf(r, 0.0f), (float)QMAX);
+      q = (int)r;
+    }
+    code[e] = q;
+  }
+  pack_codes<BITS, WHICH>(code, sub, tip, lane);
+  if ((lane & 7) == 0) {
+    reinterpret_cast<__half *>(sub + lay.d)[tip * 4 + (lane >> 3)] = dh;
+    reinterpret_cast<__half *>(sub + lay.m)[tip * 4 + (lane >> 3)] = mh;
+  }
+}
+
+// ---- kernels ---------------------------------------------------------------------------
+
+// One warp per quantized token-head of a qb_0 / qb_1 type.  Work range per sequence:
+// tokens [a, b) = [Q(n0), Q(n1)), item = token * hkv + head.
+template <int FAM, int BITS, int WHICH>
+__global__ void __launch_bounds__(256) k_spill_qb(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in) {
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (item >= W.total) return;
+  const SeqWork &s = W.s[find_seq(W, item)];
+  const int64_t local = item - s.item0;
+  const int head = (int)(local % L.hkv);
+  const int64_t p = s.a + local / L.hkv;
+  const SubLayout lay = sub_layout(FAM, BITS);
+  uint8_t *sub = subpage_ptr(L, s.seq, p / GROUP, head, WHICH);
+  float x[4];
+  load4(src_row(L, s, head, WHICH, p, in), lane, x);
+  const int tip = (int)(p % GROUP);
+  if constexpr (FAM == FAM_SYM)
+    quant_sym<BITS, WHICH>(x, sub, lay, tip, lane);
+  else
+    quant_asym<BITS, WHICH>(x, sub, lay, tip, lane);
+}
+
+constexpr int KV_THREADS = 256;
+constexpr int XS = D + 1;  // padded row stride of the fp32 tile in shared memory
+constexpr size_t KVARN_SMEM =
+    sizeof(float) * ((size_t)GROUP * XS + GROUP /*u*/ + GROUP /*t*/ + D /*c*/ + D /*w*/ + 8 * GROUP /*part*/ +
+                     D /*rc*/ + GROUP /*rt*/);
+
+// One CTA (256 threads) per (kvarn group, head).  Per sequence, s.a is the first group
+// the append touches (it may be a partial group that grows) and s.b the quantized length
+// Q(n1) after the append; items enumerate (group, head).
+template <int BITS, int WHICH>
+__global__ void __launch_bounds__(KV_THREADS, 1)
+    k_spill_kvarn(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in, int iters) {
+  extern __shared__ float sm[];
+  float *X = sm;
+  float *u = X + GROUP * XS;
+  float *tt = u + GROUP;
+  float *cj = tt + GROUP;
+  float *wj = cj + D;
+  float *part = wj + D;
+  float *rc = part + 8 * GROUP;
+  float *rt = rc + D;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t item = blockIdx.x;
+  const SeqWork &s = W.s[find_seq(W, item)];
+  const int64_t local = item - s.item0;
+  const int head = (int)(local % L.hkv);
+  const int64_t g = s.a + local / L.hkv;
+  const int64_t g0 = g * GROUP;
+  const int64_t Q1 = s.b;  // quantized length after the append
+  const int ng = (int)((Q1 - g0) < GROUP ? (Q1 - g0) : GROUP);
+  const SubLayout lay = sub_layout(FAM_KVARN, BITS);
+  uint8_t *sub = subpage_ptr(L, s.seq, g, head, WHICH);
+
+  // 1. load the group's BF16 rows (ring or new input) as fp32
+  for (int i = warp; i < ng; i += 8) {
+    float x[4];
+    load4(src_row(L, s, head, WHICH, g0 + i, in), lane, x);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) X[i * XS + 4 * lane + e] = x[e];
+  }
+  __syncthreads();
+
+  // 2. Walsh-Hadamard rotation of each row: stages h = 1..64 ascending, then times kappa
+  if (tid < ng) {
+    float r[D];
+#pragma unroll
+    for (int j = 0; j < D; ++j) r[j] = X[tid * XS + j];
+#pragma unroll
+    for (int h = 1; h < D; h <<= 1) {
+#pragma unroll
+      for (int j = 0; j < D; ++j) {
+        if (j & h) continue;
+        const float a = r[j], b = r[j + h];
+        r[j] = __fadd_rn(a, b);
+        r[j + h] = __fsub_rn(a, b);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < D; ++j) X[tid * XS + j] = __fmul_rn(r[j], kKappa());
+    tt[tid] = 1.0f;
+  }
+  __syncthreads();
+
+  // 3. Sinkhorn, scale-only form.  Thread (warp w, lane l) covers channels 16w..16w+15 and
+  //    tokens l, l+32, ..., l+224: channel sums chain over its tokens then xor-butterfly
+  //    over lanes (16, 8, 4, 2, 1); token sums chain over its 16 channels, then the 8 warp
+  //    partials are combined by an xor butterfly (4, 2, 1).
+  const float fng = (float)ng;
+  for (int it = 0; it < iters; ++it) {
+    if (tid < ng) u[tid] = __fdiv_rn(1.0f, __fmul_rn(tt[tid], tt[tid]));
+    __syncthreads();
+#pragma unroll 4
+    for (int cc = 0; cc < 16; ++cc) {
+      const int j = 16 * warp + cc;
+      float acc = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = lane + 32 * k;
+        if (i < ng) {
+          const float x = X[i * XS + j];
+          acc = __fmaf_rn(__fmul_rn(x, x), u[i], acc);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL, acc, o));
+      if (lane == 0) {
+        const float c = acc > 0.0f ? __fsqrt_rn(__fdiv_rn(acc, fng)) : 1.0f;
+        cj[j] = c;
+        wj[j] = __fdiv_rn(1.0f, __fmul_rn(c, c));
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = lane + 32 * k;
+      if (i < ng) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          const int j = 16 * warp + cc;
+          const float x = X[i * XS + j];
+          acc = __fmaf_rn(__fmul_rn(x, x), wj[j], acc);
+        }
+        part[warp * GROUP + i] = acc;
+      }
+    }
+    __syncthreads();
+    if (tid < ng) {
+      float p[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) p[r] = part[r * GROUP + tid];
+      const float a0 = __fadd_rn(p[0], p[4]), a1 = __fadd_rn(p[1], p[5]);
+      const float a2 = __fadd_rn(p[2], p[6]), a3 = __fadd_rn(p[3], p[7]);
+      const float b0 = __fadd_rn(a0, a2), b1 = __fadd_rn(a1, a3);
+      const float R = __fadd_rn(b0, b1);
+      tt[tid] = R > 0.0f ? __fsqrt_rn(__fdiv_rn(R, 128.0f)) : 1.0f;
+    }
+    __syncthreads();
+  }
+
+  // 4. fp16 scales; normalization uses the stored (fp16) values
+  if (tid < D) {
+    const __half h = scale_to_half(cj[tid]);
+    reinterpret_cast<__half *>(sub + lay.c)[tid] = h;
+    rc[tid] = __fdiv_rn(1.0f, __half2float(h));
+  }
+  if (tid < ng) {
+    const __half h = scale_to_half(tt[tid]);
+    reinterpret_cast<__half *>(sub + lay.t)[tid] = h;
+    rt[tid] = __fdiv_rn(1.0f, __half2float(h));
+  }
+  __syncthreads();
+
+  // 5. y = (x * rc_j) * rt_i, symmetric b-bit blocks of 32, packed
+  for (int i = warp; i < ng; i += 8) {
+    float y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * lane + e;
+      y[e] = __fmul_rn(__fmul_rn(X[i * XS + j], rc[j]), rt[i]);
+    }
+    quant_sym<BITS, WHICH>(y, sub, lay, i, lane);
+  }
+}
+
+// Copies new rows that stay 16-bit into the ring: range per sequence [a, n1), rows
+// enumerated as (token, head), 16 threads per 256-byte row.
+__global__ void __launch_bounds__(256) k_tail_write(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t item = t >> 4;
+  const int part = (int)(t & 15);
+  if (item >= W.total) return;
+  const SeqWork &s = W.s[find_seq(W, item)];
+  const int64_t local = item - s.item0;
+  const int head = (int)(local % L.hkv);
+  const int64_t p = s.a + local / L.hkv;
+  const uint4 *src = reinterpret_cast<const uint4 *>(in + ((s.in_off + (p - s.n0)) * L.hkv + head) * D);
+  uint4 *dst = reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, W.which, p));
+  dst[part] = src[part];
+}
+
+// ---- dispatch ----------------------------------------------------------------------------
+
+template <int WHICH>
+cudaError_t spill_qb(int fam, int bits, const LayerView &L, const Work &W, const __nv_bfloat16 *in,
+                     cudaStream_t st) {
+  const unsigned grid = (unsigned)((W.total + 7) / 8);
+#define KVQ_QB(F, B) \
+  if (fam == F && bits == B) { k_spill_qb<F, B, WHICH><<<grid, 256, 0, st>>>(L, W, in); return cudaGetLastError(); }
+  KVQ_QB(FAM_SYM, 2) KVQ_QB(FAM_SYM, 3) KVQ_QB(FAM_SYM, 4) KVQ_QB(FAM_SYM, 5) KVQ_QB(FAM_SYM, 6)
+  KVQ_QB(FAM_SYM, 8) KVQ_QB(FAM_ASYM, 2) KVQ_QB(FAM_ASYM, 3) KVQ_QB(FAM_ASYM, 4) KVQ_QB(FAM_ASYM, 5)
+  KVQ_QB(FAM_ASYM, 6)
+#undef KVQ_QB
+  return cudaErrorInvalidValue;
+}
+
+template <int BITS, int WHICH>
+cudaError_t launch_kvarn_t(const LayerView &L, const Work &W, const __nv_bfloat16 *in, int iters, cudaStream_t st) {
+  static bool attr_set = false;  // per template instance; the attribute is per function
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_spill_kvarn<BITS, WHICH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)KVARN_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  k_spill_kvarn<BITS, WHICH><<<(unsigned)W.total, KV_THREADS, KVARN_SMEM, st>>>(L, W, in, iters);
+  return cudaGetLastError();
+}
+
+template <int WHICH>
+cudaError_t spill_kvarn(int bits, const LayerView &L, const Work &W, const __nv_bfloat16 *in, int iters,
+                        cudaStream_t st) {
+  switch (bits) {
+    case 2: return launch_kvarn_t<2, WHICH>(L, W, in, iters, st);
+    case 3: return launch_kvarn_t<3, WHICH>(L, W, in, iters, st);
+    case 4: return launch_kvarn_t<4, WHICH>(L, W, in, iters, st);
+    case 5: return launch_kvarn_t<5, WHICH>(L, W, in, iters, st);
+    case 6: return launch_kvarn_t<6, WHICH>(L, W, in, iters, st);
+    case 8: return launch_kvarn_t<8, WHICH>(L, W, in, iters, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &seqs, const void *k,
+                  const void *v, cudaStream_t st) {
+  const LayerView L = layer_view(c, layer);
+  const __nv_bfloat16 *in[2] = {static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v)};
+  const int fam[2] = {c->fam_k, c->fam_v}, bits[2] = {c->bits_k, c->bits_v};
+  const int64_t hkv = c->p.n_kv_heads;
+
+  for (size_t base = 0; base < seqs.size(); base += MAXS) {
+    const size_t cnt = std::min<size_t>(MAXS, seqs.size() - base);
+    // 1. spill quantization, K then V
+    for (int which = 0; which < 2; ++which) {
+      if (fam[which] == FAM_BF16) continue;
+      Work W{};
+      W.which = which;
+      int64_t total = 0;
+      for (size_t i = 0; i < cnt; ++i) {
+        const AppendSeq &a = seqs[base + i];
+        SeqWork &s = W.s[W.n];
+        s.seq = a.seq;
+        s.n0 = a.n0;
+        s.n1 = a.n0 + a.n_new;
+        s.in_off = a.in_off;
+        const int64_t Q0 = quantized_len(c, s.n0), Q1 = quantized_len(c, s.n1);
+        if (Q1 <= Q0) continue;
+        int64_t items;
+        if (fam[which] == FAM_KVARN) {
+          s.a = Q0 / GROUP;               // first group touched (may be partial)
+          s.b = Q1;                       // quantized length after the append
+          items = ((Q1 - 1) / GROUP - s.a + 1) * hkv;
+        } else {
+          s.a = Q0;
+          s.b = Q1;
+          items = (Q1 - Q0) * hkv;
+        }
+        s.item0 = total;
+        total += items;
+        ++W.n;
+      }
+      W.total = total;
+      if (total == 0) continue;
+      cudaError_t e = fam[which] == FAM_KVARN
+                          ? (which == 0 ? spill_kvarn<0>(bits[which], L, W, in[which], c->p.sinkhorn_iters, st)
+                                        : spill_kvarn<1>(bits[which], L, W, in[which], c->p.sinkhorn_iters, st))
+                          : (which == 0 ? spill_qb<0>(fam[which], bits[which], L, W, in[which], st)
+                                        : spill_qb<1>(fam[which], bits[which], L, W, in[which], st));
+      if (e != cudaSuccess) return KVQ_E_CUDA;
+    }
+    // 2. ring write of the new rows that stay 16-bit
+    for (int which = 0; which < 2; ++which) {
+      Work W{};
+      W.which = which;
+      int64_t total = 0;
+      for (size_t i = 0; i < cnt; ++i) {
+        const AppendSeq &a = seqs[base + i];
+        SeqWork &s = W.s[W.n];
+        s.seq = a.seq;
+        s.n0 = a.n0;
+        s.n1 = a.n0 + a.n_new;
+        s.in_off = a.in_off;
+        const int64_t ks = keep_start(c, fam[which], s.n1);
+        s.a = ks > s.n0 ? ks : s.n0;
+        s.b = s.n1;
+        if (s.b <= s.a) continue;
+        s.item0 = total;
+        total += (s.b - s.a) * hkv;
+        ++W.n;
+      }
+      W.total = total;
+      if (total == 0) continue;
+      const int64_t threads = total * 16;
+      k_tail_write<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(L, W, in[which]);
+      if (cudaGetLastError() != cudaSuccess) return KVQ_E_CUDA;
+    }
+  }
+  return KVQ_OK;
+}
+
+}  // namespace kvq

@@ -1,0 +1,52 @@
+"""The C-ABI library loads without a GPU, exports every entry point include/kvq.h
+declares, and validates arguments on the host (no device call is needed for these)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    from bit_kv_cache_17_b200 import kvq
+
+    lib = C.CDLL(kvq.LIB_PATH)
+    names = declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(kvq.EXPORTED)
+
+
+def test_host_validation_and_sizes():
+    from bit_kv_cache_17_b200 import kvq
+
+    p = kvq.kvq_default_params(n_kv_heads=8, max_ctx=65536, type_k="kvarn4", type_v="kvarn4", tail=1024)
+    nb = kvq.kvq_cache_bytes(p)
+    # 256 pages x 8 heads x (K + V sub-pages of 19200 B) plus a 1280-row ring per stream
+    assert nb >= 256 * 8 * 2 * 19200 + 8 * 2 * 1280 * 256
+    for bad in (dict(head_dim=64), dict(group=128), dict(page_tokens=512)):
+        with pytest.raises(kvq.KVQError) as e:
+            kvq.kvq_cache_bytes(kvq.kvq_default_params(**bad))
+        assert e.value.code == kvq.KVQ_E_UNSUPPORTED
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.kvq_cache_bytes(kvq.kvq_default_params(type_k="bf16", type_v="q4_0"))
+    assert e.value.code == kvq.KVQ_E_UNSUPPORTED
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.kvq_cache_bytes(kvq.kvq_default_params(tail=-1))
+    assert e.value.code == kvq.KVQ_E_INVAL
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.kvq_cache_create(p, 0, nb)
+    assert e.value.code == kvq.KVQ_E_INVAL
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.kvq_cache_create(p, 8, nb)  # misaligned pointer is rejected before any device call
+    assert e.value.code == kvq.KVQ_E_ALIGN
+    assert kvq.kvq_strerror(kvq.KVQ_E_CAPACITY).startswith("sequence capacity")
