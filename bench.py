@@ -1,0 +1,532 @@
+#!/usr/bin/env python
+"""Benchmark of the mixed-precision KV-cache hot path on B200.
+
+Headline workload (one GPU): decode attention at 64k context over a kvarn4 cache with a
+1024-token BF16 tail, 8 KV heads x 128, 40 query heads, batch 1.  One step = append one
+token (tail write, spill of the oldest tail token into its kvarn group, WHT, Sinkhorn,
+quantize) + decode attention (Q rotation, split-K over the quantized pages and the tail,
+merge with the inverse rotation of the V accumulator).  Steps cycle over `--layers`
+independent layer caches (8 x 81.6 MB by default) so that every step reads its cache from
+HBM, not L2.  The metric is decode KV bytes read per second (algorithmic bytes: codes,
+scales and tail rows of every K/V stream at the step's context length).
+
+`--impl reference` times the CPU oracle (oracle/, plain C) on the same workload instead.
+Multi-GPU (torchrun): every rank runs the same workload on its own GPU (no collective on
+the data path: independent sequences / layers); rank 0 prints the max-over-ranks time.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn KV GB/s (% of HBM peak) at 64k ctx; append Mtok/s; vs CPU oracle"
+D = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=512)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--type", default="kvarn4")
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--quick", action="store_true", help="skip the per-type sweep and the append workload")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------
+# algorithmic bytes
+
+def decode_bytes(calc, type_, n, tail, hkv, hq):
+    """Algorithmic bytes of one decode step at context n: every K/V stream once (packed codes,
+    fp16 scales, kvarn channel scales, BF16 tail rows) plus q in and out (fp32).  `calc` is
+    a payload calculator: the library's (our arm) or the oracle's (reference arm)."""
+    per_stream = calc.payload_bytes(type_, 1, 1, n, tail) / 2.0
+    return 2 * hkv * per_stream + 2 * hq * D * 4
+
+
+class LibCalc:
+    """The library's host-only payload calculator (kvq_payload_bytes)."""
+
+    def __init__(self, kvq):
+        self.kvq = kvq
+
+    def payload_bytes(self, type_, n_layers, n_kv_heads, n, tail):
+        return self.kvq.kvq_payload_bytes(type_, n_layers, n_kv_heads, n, tail)
+
+
+# ---------------------------------------------------------------------------------------
+# clocks
+
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 10:
+                    continue
+                try:
+                    rows.append(dict(sm=float(c[2]), smax=float(c[3]), power=float(c[4]), hw=c[6], hwt=c[7],
+                                     swt=c[8], swp=c[9]))
+                except ValueError:
+                    continue
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        reasons = set()
+        for r in rows:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                            ("swp", "sw_power_cap")):
+                if r[k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; measurement only, no data-path collective)
+
+def dist_init(args):
+    import torch
+
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        if torch.cuda.is_available():
+            torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(ws, x):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------
+# our implementation
+
+def dev_bf16(torch, bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def build_decode_workload(torch, kvq, cfg, type_, layers, tokens_per_layer):
+    """Cache with `layers` layer copies of the 64k workload, each prefilled to
+    n - tokens_per_layer tokens; returns the cache and device inputs."""
+    n, hkv, hq, tail = cfg["n"], cfg["hkv"], cfg["hq"], cfg["tail"]
+    cache = kvq.KVCache(n_layers=layers, n_seqs=1, n_kv_heads=hkv, max_ctx=n, type_k=type_, type_v=type_,
+                        tail=tail)
+    from bit_kv_cache_17_b200 import synth
+
+    kt = dev_bf16(torch, synth.token_major(cfg["k"]))
+    vt = dev_bf16(torch, synth.token_major(cfg["v"]))
+    P = n - tokens_per_layer
+    for l in range(layers):
+        cache.append(l, [0], [P], kt[:P], vt[:P])
+    torch.cuda.synchronize()
+    return cache, kt, vt, P
+
+
+def run_ours(args, ws, rank):
+    import torch
+
+    from bit_kv_cache_17_b200 import kvq, synth
+
+    calc = LibCalc(kvq)
+    cfg = synth.config2()
+    hkv, hq, tail, n = cfg["hkv"], cfg["hq"], cfg["tail"], cfg["n"]
+    L = args.layers
+    W, K = args.warmup, args.steps
+    K_e2e = max(8, min(K, 256))
+    per_layer = math.ceil((W + K + K_e2e) / L)
+    assert per_layer <= 4096, "too many steps for the 64k context window"
+    cache, kt, vt, P = build_decode_workload(torch, kvq, cfg, args.type, L, per_layer)
+    qdev = torch.from_numpy(cfg["q"][:, 0]).cuda()  # [128, hq, 128]
+    out = torch.empty((W + K, 1, hq, D), dtype=torch.float32, device="cuda")
+    cache.workspace(1, hq)
+
+    def step(s, out_row):
+        layer, tok = s % L, P + s // L
+        cache.append(layer, [0], [1], kt[tok:tok + 1], vt[tok:tok + 1])
+        cache.decode(layer, [0], qdev[s % qdev.shape[0]][None], out=out_row)
+
+    def ctx(s):
+        return P + s // L + 1
+
+    # warm-up steps run eagerly (first launches set kernel attributes), then the timed
+    # steps are captured into CUDA graphs and replayed once
+    for s in range(W):
+        step(s, out[s])
+    torch.cuda.synchronize()
+    launches0 = kvq.kvq_launch_count()
+    graphs = []
+    chunk = 1024
+    for c0 in range(W, W + K, chunk):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for s in range(c0, min(W + K, c0 + chunk)):
+                step(s, out[s])
+        graphs.append(g)
+    launches = kvq.kvq_launch_count() - launches0
+
+    # decode-only graph (state unchanged) for the kernel's own duration and a clock soak
+    dec_out = torch.empty((1, hq, D), dtype=torch.float32, device="cuda")
+    gd = torch.cuda.CUDAGraph()
+    ND = 64
+    with torch.cuda.graph(gd):
+        for i in range(ND):
+            cache.decode(i % L, [0], qdev[i % qdev.shape[0]][None], out=dec_out)
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    sampler = ClockSampler("GPU-" + str(props.uuid))
+    sampler.start()
+    # soak ~1 s so that the clocks sampled below describe a GPU under this load
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        gd.replay()
+        torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 20
+    e0.record()
+    for _ in range(reps):
+        gd.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    dec_ms = e0.elapsed_time(e1) / (reps * ND)
+
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for g in graphs:
+        g.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = t0.elapsed_time(t1)
+    clocks = sampler.stop()
+    ms_max = max_over_ranks(ws, ms)
+
+    bytes_steps = sum(decode_bytes(calc, args.type, ctx(s), tail, hkv, hq) for s in range(W, W + K))
+    value = ws * bytes_steps / (ms_max * 1e-3) / 1e9
+    dec_bytes = decode_bytes(calc, args.type, ctx(W + K - 1), tail, hkv, hq)
+    assert cache.status() == 0
+
+    # end to end through the public API with host buffers: H2D of the step's token K/V and
+    # q from pinned memory, append, decode, D2H of the output, every step
+    hk = torch.from_numpy(synth.token_major(cfg["k"])[P:].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(synth.token_major(cfg["v"])[P:].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hq_host = torch.from_numpy(cfg["q"][:, 0]).pin_memory()
+    hout = torch.empty((K_e2e, 1, hq, D), dtype=torch.float32).pin_memory()
+    dk = torch.empty((1, hkv, D), dtype=torch.bfloat16, device="cuda")
+    dv = torch.empty_like(dk)
+    dq = torch.empty((1, hq, D), dtype=torch.float32, device="cuda")
+    do = torch.empty_like(dq)
+    s0 = W + K
+    barrier(ws)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for j in range(K_e2e):
+        s = s0 + j
+        layer, tok = s % L, s // L
+        dk.copy_(hk[tok:tok + 1], non_blocking=True)
+        dv.copy_(hv[tok:tok + 1], non_blocking=True)
+        dq.copy_(hq_host[s % hq_host.shape[0]][None], non_blocking=True)
+        cache.append(layer, [0], [1], dk, dv)
+        cache.decode(layer, [0], dq, out=do)
+        hout[j].copy_(do, non_blocking=True)
+    a1.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e2e_ms = max_over_ranks(ws, a0.elapsed_time(a1))
+    e2e_bytes = sum(decode_bytes(calc, args.type, ctx(s0 + j), tail, hkv, hq) for j in range(K_e2e))
+    e2e = {"value": round(ws * e2e_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": int(2 * hkv * D * 2 + hq * D * 4), "d2h_bytes_per_step": int(hq * D * 4),
+           "steps": K_e2e, "ms_per_step": round(e2e_ms / K_e2e, 4)}
+
+    peaks = load_peaks()
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    roof = {"kernel": "k_decode (split-K decode + merge)", "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "peak_source": peaks["source"], "avg_launch_us": round(dec_ms * 1e3, 2),
+            "bytes_per_launch": int(dec_bytes), "traffic": traffic_for("decode", args.type)}
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded AR(1) K/V, N(0,1) queries; see bit_kv_cache_17_b200/synth.py)",
+        "config": {"workload": f"decode @64k: {args.type}, context {P + 1}..{ctx(W + K - 1)}, tail {tail} BF16, "
+                               f"{hkv} KV heads x 128, {hq} query heads, batch 1, 1 token appended per step",
+                   "layer_caches_cycled": L, "hbm_frac_of_peak": round(value / ws / peaks["hbm_gbs"], 4),
+                   "l2": f"inputs larger than L2: {L} layer caches x {dec_bytes / 1e6:.1f} MB cycled",
+                   "parallelism": f"weak: {ws} independent replicas, no collective on the data path"},
+        "roofline": roof, "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,
+    }
+    del graphs, gd
+    return result, cfg, cache
+
+
+def run_type_sweep(args, kvq, torch, synth, cfg):
+    calc = LibCalc(kvq)
+    out = {}
+    for t in ("kvarn2", "kvarn3", "kvarn4", "kvarn5", "kvarn6", "kvarn8", "q4_0", "bf16"):
+        L = args.layers
+        cache, kt, vt, P = build_decode_workload(torch, kvq, cfg, t, L, 1)
+        # fill the last token so that every layer holds exactly 65536 tokens
+        for l in range(L):
+            cache.append(l, [0], [1], kt[P:P + 1], vt[P:P + 1])
+        qdev = torch.from_numpy(cfg["q"][0, 0]).cuda()[None]
+        o = torch.empty_like(qdev)
+        cache.workspace(1, cfg["hq"])
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(4 * L):
+                cache.decode(i % L, [0], qdev, out=o)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (40 * L)
+        b = decode_bytes(calc, t, cfg["n"], cfg["tail"] if t != "bf16" else 0, cfg["hkv"], cfg["hq"])
+        out[t] = {"decode_us": round(us, 2), "GB_per_s": round(b / us / 1e3, 1), "bytes": int(b)}
+        del cache, g
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_append(args, kvq, torch, synth):
+    """Batched prefill-append: 16 sequences built to L_i ~ U[4096, 32768], then one timed
+    append of 4096 tokens per sequence (kvarn4, tail 1024)."""
+    cfg = synth.config3(steps=0)
+    hkv, tail = cfg["hkv"], cfg["tail"]
+    Ls = cfg["lengths"]
+    S = len(Ls)
+    cache = kvq.KVCache(n_layers=1, n_seqs=S, n_kv_heads=hkv, max_ctx=max(Ls) + cfg["prefill"] + 64,
+                        type_k="kvarn4", type_v="kvarn4", tail=tail)
+    ks = [dev_bf16(torch, synth.token_major(k)) for k in cfg["k"]]
+    vs = [dev_bf16(torch, synth.token_major(v)) for v in cfg["v"]]
+    cache.append(0, list(range(S)), Ls, torch.cat([k[:l] for k, l in zip(ks, Ls)]),
+                 torch.cat([v[:l] for v, l in zip(vs, Ls)]))
+    P = cfg["prefill"]
+    kin = torch.cat([k[l:l + P] for k, l in zip(ks, Ls)])
+    vin = torch.cat([v[l:l + P] for v, l in zip(vs, Ls)])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cache.append(0, list(range(S)), [P] * S, kin, vin)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert cache.status() == 0
+    # algorithmic bytes: new rows in, the old tail + open-group rows re-read, quantized
+    # tokens and the new tail out (per stream)
+    tb = 75.0
+    moved = 0.0
+    for l in Ls:
+        q0 = l - tail
+        q1 = l + P - tail
+        staged = q0 - (q0 // 256) * 256
+        moved += 2 * hkv * (P * 256 + (tail + staged) * 256 + (q1 - (q0 // 256) * 256) * tb + tail * 256)
+    return {"metric": "append Mtok/s", "value": round(S * P / (ms * 1e-3) / 1e6, 2), "unit": "Mtok/s",
+            "ms": round(ms, 4), "GB_per_s": round(moved / (ms * 1e-3) / 1e9, 1), "bytes": int(moved),
+            "workload": f"{S} sequences, lengths {min(Ls)}..{max(Ls)}, +{P} tokens each in one call, kvarn4, "
+                        f"tail {tail}, 8 KV heads x 128"}
+
+
+# ---------------------------------------------------------------------------------------
+# measured peaks and committed ncu traffic
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured (MEASURED_PEAKS.json)"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def traffic_for(kernel, type_):
+    """dram bytes per launch from the committed ncu summary, or None when the kernel source
+    changed since the counters were taken."""
+    import hashlib
+
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(f"{kernel}:{type_}")
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "bit_kv_cache_17_b200", "csrc", ent["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return ent["dram_bytes_per_launch"] if h == ent["source_sha256_16"] else None
+
+
+# ---------------------------------------------------------------------------------------
+# the CPU oracle
+
+def oracle_decode_sample(cfg, type_, heads, n):
+    """Times the oracle's decode (stream state rebuilt from the BF16 history, fp64
+    dequant + attention) for `heads` KV heads of one step at context n."""
+    import oracle
+
+    G = cfg["hq"] // cfg["hkv"]
+    q = cfg["q"][0, 0]
+    t0 = time.perf_counter()
+    for h in heads:
+        oracle.decode_head(type_, type_, cfg["k"][h, :n], cfg["v"][h, :n], cfg["tail"], q[h * G:(h + 1) * G])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, type_):
+    import oracle as calc
+
+    n = cfg["n"]
+    heads = [0, 1, 2, 3]
+    dt = oracle_decode_sample(cfg, type_, heads, n)
+    b = decode_bytes(calc, type_, n, cfg["tail"], len(heads), len(heads) * cfg["hq"] // cfg["hkv"])
+    return {"value": round(b / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"one decode step of 1 of {cfg['hkv']} KV heads at context {n} ({type_}), "
+                      f"{dt:.1f} s single-threaded; the oracle rebuilds the stream state from BF16 each call"}
+
+
+def run_reference(args, ws, rank):
+    """The CPU oracle as the reference arm.  Each step is a bounded sample of the workload:
+    the decode of one KV head over a 4096-token window of its 64k stream (3072 quantized
+    tokens + the 1024-token BF16 tail), windows and heads cycling, so that the whole run
+    ends within minutes on one core."""
+    import oracle
+    from bit_kv_cache_17_b200 import synth
+
+    calc = oracle
+    cfg = synth.config2()
+    win, hkv, G = 4096, cfg["hkv"], cfg["hq"] // cfg["hkv"]
+    q = cfg["q"][0, 0]
+    steps = []
+    for s in range(args.warmup + args.steps):
+        h = s % hkv
+        a = (s // hkv * win) % (cfg["n"] - win)
+        a -= a % 256
+        t0 = time.perf_counter()
+        oracle.decode_head(args.type, args.type, cfg["k"][h, a:a + win], cfg["v"][h, a:a + win], cfg["tail"],
+                           q[h * G:(h + 1) * G])
+        if s >= args.warmup:
+            steps.append(time.perf_counter() - t0)
+    b = decode_bytes(calc, args.type, win, cfg["tail"], 1, G)
+    tot = sum(steps)
+    value = b * len(steps) / tot / 1e9
+    sample = (f"each step: decode of 1 of {hkv} KV heads over a {win}-token window (3072 {args.type} + 1024 BF16 "
+              f"tail) of the 64k stream, single-threaded C oracle")
+    return {"metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(tot / len(steps) * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"decode @64k: {args.type}, context {cfg['n']}, tail {cfg['tail']} BF16, "
+                                   f"{hkv} KV heads x 128, {cfg['hq']} query heads, batch 1"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        print(json.dumps(run_reference(args, ws, rank)))
+        return 0
+    ws, rank, local = dist_init(args)
+    import torch
+
+    from bit_kv_cache_17_b200 import kvq, synth
+
+    result, cfg, cache = run_ours(args, ws, rank)
+    del cache
+    torch.cuda.empty_cache()
+    if not args.quick:
+        result["per_type_decode_64k"] = run_type_sweep(args, kvq, torch, synth, cfg)
+        torch.cuda.empty_cache()
+        result["append"] = run_append(args, kvq, torch, synth)
+    if rank == 0 and ws == 1:
+        result["cpu_baseline"] = cpu_baseline(cfg, args.type)
+    elif rank == 0:
+        result["cpu_baseline"] = None
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <new>
 #include <string>
 #include <vector>
@@ -75,6 +76,9 @@ size_t plan(kvq_cache *c) {
 }  // namespace
 
 namespace kvq {
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
 LayerView layer_view(const kvq_cache *c, int layer) {
   LayerView L;
   L.pages = c->base + c->off_pages + c->layer_pages_bytes * layer;
@@ -310,6 +314,12 @@ const char *kvq_describe(kvq_cache *c) {
            c->layer_pages_bytes, c->layer_ring_bytes);
   c->desc = buf;
   return c->desc.c_str();
+}
+
+int kvq_launch_count(uint64_t *count) {
+  if (!count) return KVQ_E_INVAL;
+  *count = g_launches.load(std::memory_order_relaxed);
+  return KVQ_OK;
 }
 
 const char *kvq_strerror(int code) {

@@ -454,6 +454,7 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
                           : (which == 0 ? spill_qb<0>(fam[which], bits[which], L, W, in[which], st)
                                         : spill_qb<1>(fam[which], bits[which], L, W, in[which], st));
       if (e != cudaSuccess) return KVQ_E_CUDA;
+      note_launches(1);
     }
     // 2. ring write of the new rows that stay 16-bit
     for (int which = 0; which < 2; ++which) {
@@ -480,6 +481,7 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
       const int64_t threads = total * 16;
       k_tail_write<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(L, W, in[which]);
       if (cudaGetLastError() != cudaSuccess) return KVQ_E_CUDA;
+      note_launches(1);
     }
   }
   return KVQ_OK;

@@ -454,6 +454,7 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
     A.ncta = cta;
     // q / out rows are indexed by DecodeSeq::row, the workspace slots restart per launch
     if (dispatch(c->fam_k, c->bits_k, L, A, st) != cudaSuccess) return KVQ_E_CUDA;
+    note_launches(1);
   }
   return KVQ_OK;
 }

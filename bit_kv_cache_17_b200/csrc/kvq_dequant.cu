@@ -95,7 +95,7 @@ int launch_dequant(const kvq_cache *c, int layer, int seq, int which, int64_t t0
   const unsigned grid = (unsigned)((items + 7) / 8);
 #define KVQ_DQ(F, B) \
   if (fam == F && bits == B) { k_dequant<F, B><<<grid, 256, 0, st>>>(L, seq, which, t0, t1, Q, basis, out); \
-    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_E_CUDA; }
+    note_launches(1); return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_E_CUDA; }
   KVQ_DQ(FAM_BF16, 16)
   KVQ_DQ(FAM_SYM, 2) KVQ_DQ(FAM_SYM, 3) KVQ_DQ(FAM_SYM, 4) KVQ_DQ(FAM_SYM, 5) KVQ_DQ(FAM_SYM, 6) KVQ_DQ(FAM_SYM, 8)
   KVQ_DQ(FAM_ASYM, 2) KVQ_DQ(FAM_ASYM, 3) KVQ_DQ(FAM_ASYM, 4) KVQ_DQ(FAM_ASYM, 5) KVQ_DQ(FAM_ASYM, 6)

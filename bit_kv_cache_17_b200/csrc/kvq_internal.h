@@ -30,6 +30,9 @@ struct kvq_cache {
 
 namespace kvq {
 
+// Counts kernel launches (kvq_launch_count).
+void note_launches(int n);
+
 // Tokens of a stream kept in the BF16 ring after it holds n tokens: [keep_start, n).
 // qb types keep the tail; kvarn also keeps the rows of its open (partial) group.
 inline int64_t quantized_len(const kvq_cache *c, int64_t n) {

@@ -56,6 +56,7 @@ _SIG = {
     "kvq_get_status": (C.c_int, [_vp, _vp]),
     "kvq_describe": (C.c_char_p, [_vp]),
     "kvq_strerror": (C.c_char_p, [C.c_int]),
+    "kvq_launch_count": (C.c_int, [C.POINTER(C.c_uint64)]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -151,6 +152,12 @@ def kvq_locate(h, kind, layer, seq, page, head, which, token=0):
 
 def kvq_get_status(h, stream=0):
     return _lib.kvq_get_status(h, _vp(stream))
+
+
+def kvq_launch_count():
+    n = C.c_uint64()
+    _check(_lib.kvq_launch_count(C.byref(n)), "kvq_launch_count")
+    return n.value
 
 
 def kvq_describe(h):

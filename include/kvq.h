@@ -170,6 +170,10 @@ const char *kvq_describe(kvq_cache *c);
 
 const char *kvq_strerror(int code);
 
+/* Diagnostic: number of kernels this library has launched (or recorded into a CUDA graph
+ * under stream capture) in this process, across all caches. */
+int kvq_launch_count(uint64_t *count);
+
 #ifdef __cplusplus
 }
 #endif
