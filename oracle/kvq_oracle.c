@@ -365,7 +365,7 @@ int64_t kvqo_stream_state(int type, const uint16_t *xb, int64_t n, int64_t tail,
 }
 
 /* ------------------------------------------------------------------------------------ */
-/* packing (the pages fix no bit layout; the layout below is this build's definition)  */
+/* packing (the pages fix no bit layout; the layout below is the definition used)      */
 /* ------------------------------------------------------------------------------------ */
 
 /* b-bit codes are split into a low plane of width wlo and a high plane of width whi. */

@@ -16,10 +16,10 @@
  *        Walsh-Hadamard transform and Sinkhorn save quality at 4-bit".
  *   [p5] molayo1419.me, "BeeLLama.cpp v0.4.0: KVarN, precision tail, q2_0-q3_1"
  *        - KLD table (cache types kvarn2..kvarn8).
- * The pages give KVarN only qualitatively; the task specification fixes its steps
- * (Sylvester Hadamard in a fixed fp32 butterfly order, 8 Sinkhorn iterations,
- * fp16 per-channel and per-token scales, symmetric blocks of 32 with fp16 d).
- * Every reading taken where that is still open is listed in the design doc.
+ * The pages give KVarN only qualitatively.  Its steps are fixed here as: Sylvester
+ * Hadamard rotation in a fixed fp32 butterfly order, 8 Sinkhorn iterations into fp16
+ * per-channel and per-token scales, symmetric blocks of 32 with an fp16 scale d.  Where
+ * the pages leave a step open, the comment at the step states the reading taken.
  *
  * Parity status per function (see the header of kvq_oracle.c for the pins):
  *   every exported function below is pinned by at least one test in

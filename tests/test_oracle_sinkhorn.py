@@ -1,6 +1,6 @@
 """Pins of the oracle's Sinkhorn balancing (Bonsai-Ternary-27B page, "How the WHT and
 Sinkhorn save quality": a per-dimension scale equalizes the spread before quantizing;
-the task fixes 8 iterations of channel-RMS then token-RMS division into fp16 scales)."""
+the steps used are 8 iterations of channel-RMS then token-RMS division into fp16 scales)."""
 import numpy as np
 
 import oracle
