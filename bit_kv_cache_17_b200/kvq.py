@@ -57,6 +57,7 @@ _SIG = {
     "kvq_describe": (C.c_char_p, [_vp]),
     "kvq_strerror": (C.c_char_p, [C.c_int]),
     "kvq_launch_count": (C.c_int, [C.POINTER(C.c_uint64)]),
+    "kvq_decode_attn_noalloc": (C.c_int, [_vp, _i32, _i32, C.POINTER(_i32), _i32, _vp, C.c_float, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -128,6 +129,12 @@ def kvq_decode_attn(h, layer, seq_ids, n_q_heads, q_ptr, softmax_scale, out_ptr,
     rc = _lib.kvq_decode_attn(h, layer, len(seq_ids), _i32arr(seq_ids), n_q_heads, _vp(q_ptr), softmax_scale,
                               _vp(out_ptr), _vp(ws_ptr), ws_bytes, _vp(stream))
     _check(rc, "kvq_decode_attn")
+
+
+def kvq_decode_attn_noalloc(h, layer, seq_ids, n_q_heads, q_ptr, softmax_scale, out_ptr, stream=0):
+    rc = _lib.kvq_decode_attn_noalloc(h, layer, len(seq_ids), _i32arr(seq_ids), n_q_heads, _vp(q_ptr), softmax_scale,
+                                      _vp(out_ptr), _vp(stream))
+    _check(rc, "kvq_decode_attn_noalloc")
 
 
 def kvq_dequant(h, layer, seq, which, t0, t1, basis, out_ptr, stream=0):

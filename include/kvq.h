@@ -170,6 +170,26 @@ const char *kvq_describe(kvq_cache *c);
 
 const char *kvq_strerror(int code);
 
+/* Decode attention that allocates nothing: the same computation and arguments as
+ * kvq_decode_attn, without the workspace.  The pages have no counterpart of this entry
+ * point; it exists for callers that cannot allocate device memory: a plugin running inside
+ * a host runtime that owns all device memory and offers it no allocator, or a serving loop
+ * that must not allocate (a possible stall or failure) once it runs.
+ *  - The split-K partial results go to one library-owned static device array of
+ *    KVQ_NOALLOC_SCRATCH_BYTES (4 MiB) per GPU, held by every GPU that loads the library
+ *    until the process exits.  A call whose partials need more (kvq_workspace_bytes for
+ *    the same n_seqs / n_q_heads) returns KVQ_E_SIZE and launches nothing.
+ *  - The first call on a device looks up the array's device address (with that device
+ *    current) and keeps it; make that first call before any stream capture.
+ *  - Every call shares the array and it keeps the last call's contents; nothing in it needs
+ *    to start at zero (every partial is written before it is read).  Calls that overlap on
+ *    the GPU, on any stream or cache, race on the array: issue them in stream order.
+ *  - Never calls cudaMalloc, cudaFree or any allocating routine. */
+#define KVQ_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+int kvq_decode_attn_noalloc(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,
+                            int32_t n_q_heads, const float *q, float softmax_scale, float *out,
+                            kvq_stream_t stream);
+
 /* Diagnostic: number of kernels this library has launched (or recorded into a CUDA graph
  * under stream capture) in this process, across all caches. */
 int kvq_launch_count(uint64_t *count);
