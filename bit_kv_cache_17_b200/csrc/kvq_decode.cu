@@ -23,7 +23,7 @@ namespace kvq {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int DT = 128;      // threads per CTA
+constexpr int DT = 256;      // threads per CTA (one CTA per SM)
 constexpr int NW = DT / 32;  // warps per CTA
 constexpr int CH = 32;       // tokens per chunk (one per lane)
 constexpr int MAXSQ = 48;    // max splits over the quantized prefix per (seq, head)
@@ -63,32 +63,614 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// field of channel ch of a K token held as 32-bit words (indices resolve at compile time)
-template <int BITS>
-__device__ __forceinline__ uint32_t k_field_w(const uint32_t *w, int ch) {
-  constexpr int WL = plane_lo(BITS), WH = plane_hi(BITS);
-  const int blk = ch >> 5, e = ch & 31, jj = e >> 2, k = e & 3;
-  constexpr int FL = 8 / WL;
-  const int bl = 16 * (jj / FL) + 4 * blk + k;
-  uint32_t f = (w[bl >> 2] >> (8 * (bl & 3) + (jj % FL) * WL)) & ((1u << WL) - 1u);
-  if constexpr (WH > 0) {
-    constexpr int FH = 8 / WH;
-    const int bh = 16 * WL + 16 * (jj / FH) + 4 * blk + k;
-    f |= ((w[bh >> 2] >> (8 * (bh & 3) + (jj % FH) * WH)) & ((1u << WH) - 1u)) << WL;
+// ---- tensor-core pieces (mma.sync m16n8k32, s8 x s8 -> s32) ---------------------------
+//
+// Fragment layout (groupID g = lane/4, thread-in-group tq = lane%4):
+//   A 16x32: a0 = (row g, k 4tq..4tq+3), a1 = (row g+8, same k), a2 = (row g, k 16+4tq..),
+//            a3 = (row g+8, k 16+4tq..);  B 32x8: b0 = (k 4tq.., col g), b1 = (k 16+4tq.., col g);
+//   C 16x8: c0 = (row g, col 2tq), c1 = (g, 2tq+1), c2 = (g+8, 2tq), c3 = (g+8, 2tq+1).
+// Rows 0..7 carry the high int8 limb and rows 8..15 the low limb of a 16-bit fixed-point
+// operand of query head g (Q for Q.K, the softmax weights for P.V); both MMA results of one
+// column combine exactly in int32 as 256*hi + lo.
+
+__device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// field s (width W) of each byte of `word`, moved to bits [P, P+W) of the same byte
+template <int W, int P>
+__device__ __forceinline__ uint32_t xplane(uint32_t word, int s) {
+  constexpr uint32_t M1 = ((1u << W) - 1u) << P;
+  constexpr uint32_t M = M1 | (M1 << 8) | (M1 << 16) | (M1 << 24);
+  return __funnelshift_l(word, word, (P - s * W) & 31) & M;
+}
+
+__device__ __forceinline__ uint32_t wsel(const uint4 &v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+__device__ __forceinline__ uint4 ld16(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
+
+// K codes of one token, as the B fragment of block blk: reg e holds channels
+// 32 blk + 8 tq + 4 e + (0..3) as bytes code * 2^(8-b) (signed) or (u - 2^(b-1)) * 2^(8-b).
+template <int FAM, int BITS>
+struct KTok {
+  static constexpr int WL = plane_lo(BITS), WH = plane_hi(BITS);
+  uint4 l0, l1, h0;
+  __device__ __forceinline__ void load(const uint8_t *tok, int tq) {
+    if constexpr (WL == 8) {
+      l0 = ld16(tok + 32 * tq);
+      l1 = ld16(tok + 32 * tq + 16);
+    } else if constexpr (WL == 4) {
+      l0 = ld16(tok + 16 * tq);
+    } else {
+      l0 = ld16(tok + 16 * (tq >> 1));
+    }
+    if constexpr (WH == 1) h0 = ld16(tok + 16 * WL);
+    if constexpr (WH == 2) h0 = ld16(tok + 16 * WL + 16 * (tq >> 1));
   }
-  return f;
+  __device__ __forceinline__ void frag(int blk, int tq, uint32_t &b0, uint32_t &b1) const {
+    constexpr int PL = 8 - BITS;
+    const uint32_t w0 = wsel(l0, blk);
+    if constexpr (WL == 8) {
+      b0 = w0;
+      b1 = wsel(l1, blk);
+    } else if constexpr (WL == 4) {
+      b0 = xplane<4, PL>(w0, 0);
+      b1 = xplane<4, PL>(w0, 1);
+    } else {
+      const int s0 = (2 * tq) & 3;
+      b0 = xplane<2, PL>(w0, s0);
+      b1 = xplane<2, PL>(w0, s0 + 1);
+    }
+    if constexpr (WH > 0) {
+      constexpr int PH = 8 - BITS + WL, FH = 8 / WH;
+      const uint32_t wh = wsel(h0, blk);
+      const int s0 = (2 * tq) % FH;
+      b0 |= xplane<WH, PH>(wh, s0);
+      b1 |= xplane<WH, PH>(wh, s0 + 1);
+    }
+    if constexpr (FAM == FAM_ASYM) {
+      b0 ^= 0x80808080u;
+      b1 ^= 0x80808080u;
+    }
+  }
+};
+
+// V codes of one quad and one block, as B fragments for channels 32 blk + 4 g + u (u = 0..3):
+// byte k = quad token k.
+template <int FAM, int BITS>
+struct VQuad {
+  static constexpr int WL = plane_lo(BITS), WH = plane_hi(BITS);
+  uint4 l;
+  uint32_t h;
+  __device__ __forceinline__ void load(const uint8_t *quad, int blk, int g) {
+    if constexpr (WL == 8) {
+      l = ld16(quad + 128 * blk + 16 * g);
+    } else if constexpr (WL == 4) {
+      const uint2 t = *reinterpret_cast<const uint2 *>(quad + 64 * blk + 8 * g);
+      l.x = t.x;
+      l.y = t.y;
+    } else {
+      l.x = *reinterpret_cast<const uint32_t *>(quad + 32 * blk + 4 * g);
+    }
+    if constexpr (WH == 1) h = *reinterpret_cast<const uint32_t *>(quad + 64 * WL + 16 * blk + 4 * (g >> 1));
+    if constexpr (WH == 2) h = *reinterpret_cast<const uint32_t *>(quad + 64 * WL + 32 * blk + 4 * g);
+  }
+  __device__ __forceinline__ uint32_t frag(int u, int g) const {
+    constexpr int PL = 8 - BITS;
+    uint32_t r;
+    if constexpr (WL == 8)
+      r = wsel(l, u);
+    else if constexpr (WL == 4)
+      r = xplane<4, PL>(u < 2 ? l.x : l.y, u & 1);
+    else
+      r = xplane<2, PL>(l.x, u);
+    if constexpr (WH == 1) r |= xplane<1, 8 - BITS + WL>(h, 4 * (g & 1) + u);
+    if constexpr (WH == 2) r |= xplane<2, 8 - BITS + WL>(h, u);
+    if constexpr (FAM == FAM_ASYM) r ^= 0x80808080u;
+    return r;
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_s8(int a, int b, int c, int d) {
+  return (uint32_t)(a & 255) | ((uint32_t)(b & 255) << 8) | ((uint32_t)(c & 255) << 16) | ((uint32_t)(d & 255) << 24);
+}
+
+__device__ __forceinline__ float h2f(const __half *p, int i) { return __half2float(p[i]); }
+
+constexpr float QFIX = 32639.0f;              // 16-bit fixed point: 256*127 + 127
+constexpr float MAGIC = 12582912.0f + 128.0f;  // 1.5*2^23 (+128 offset for the limb split)
+
+// ---- TMA bulk copies + mbarriers (one pipeline per warp) ---------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// global -> shared bulk copy (TMA, no multicast) completing on an mbarrier; 16-byte aligned
+// addresses, size a multiple of 16
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+constexpr uint32_t kWaitLimit = 1u << 24;  // try_wait rounds before a wait is declared stuck
+constexpr int32_t kStatusWaitTimeout = 1;   // device status bit: a pipeline wait gave up
+
+// Bounded wait for a phase of an mbarrier; on timeout records the status bit and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicOr(status, kStatusWaitTimeout);
+  return false;
+}
+
+// Shared-memory image of one 32-token chunk of a quantized page (both K and V), filled by
+// bulk copies: codes of K, codes of V one quad per row with a 32-byte pad (so that the
+// lanes of one P.V fragment load hit distinct banks), then the fp16 scales.
+template <int FAM, int BITS>
+struct Stage {
+  static constexpr int QS = 64 * BITS + 32;  // padded quad stride
+  static constexpr int KC = 0;
+  static constexpr int VC = KC + 512 * BITS;
+  static constexpr int KD = VC + 8 * QS;
+  static constexpr int VD = KD + 256;
+  static constexpr int KM = VD + 256;
+  static constexpr int VM = KM + (FAM == FAM_ASYM ? 256 : 0);
+  static constexpr int KT = VM + (FAM == FAM_ASYM ? 256 : 0);
+  static constexpr int VT = KT + (FAM == FAM_KVARN ? 64 : 0);
+  static constexpr int KCS = VT + (FAM == FAM_KVARN ? 64 : 0);
+  static constexpr int VCS = KCS + (FAM == FAM_KVARN ? 256 : 0);
+  static constexpr int BYTES = VCS + (FAM == FAM_KVARN ? 256 : 0);
+  static constexpr uint32_t TX = BYTES - 8 * 32;  // bytes the copies deliver (no pads)
+  static constexpr int NST = BITS <= 3 ? 4 : (BITS <= 5 ? 3 : 2);  // stages per warp
+};
+
+// Issues the bulk copies of chunk [i0, i0+32) of page `page` into `st` (one lane).
+template <int FAM, int BITS>
+__device__ __forceinline__ void issue_chunk(const LayerView &L, int seq, int head, int64_t i0, uint8_t *st,
+                                            uint64_t *bar) {
+  using S = Stage<FAM, BITS>;
+  const SubLayout lay = sub_layout(FAM, BITS);
+  const int64_t page = i0 / GROUP;
+  const int tip0 = (int)(i0 % GROUP);
+  const uint8_t *sk = subpage_ptr(L, seq, page, head, 0);
+  const uint8_t *sv = subpage_ptr(L, seq, page, head, 1);
+  mbar_expect_tx(bar, S::TX);
+  bulk_g2s(st + S::KC, sk + tip0 * 16 * BITS, 512 * BITS, bar);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) bulk_g2s(st + S::VC + q * S::QS, sv + (tip0 / 4 + q) * 64 * BITS, 64 * BITS, bar);
+  bulk_g2s(st + S::KD, sk + lay.d + tip0 * 8, 256, bar);
+  bulk_g2s(st + S::VD, sv + lay.d + tip0 * 8, 256, bar);
+  if constexpr (FAM == FAM_ASYM) {
+    bulk_g2s(st + S::KM, sk + lay.m + tip0 * 8, 256, bar);
+    bulk_g2s(st + S::VM, sv + lay.m + tip0 * 8, 256, bar);
+  }
+  if constexpr (FAM == FAM_KVARN) {
+    bulk_g2s(st + S::KT, sk + lay.t + tip0 * 2, 64, bar);
+    bulk_g2s(st + S::VT, sv + lay.t + tip0 * 2, 64, bar);
+    bulk_g2s(st + S::KCS, sk + lay.c, 256, bar);
+    bulk_g2s(st + S::VCS, sv + lay.c, 256, bar);
+  }
+}
+
+// Q.K and P.V of one warp over its chunks [c0, c1) of a quantized split starting at token a
+// (chunks are consecutive, so pages change rarely).  Writes the warp's online-softmax state
+// (m, l and the accumulator in the stored basis) of its heads to shared memory.
+template <int FAM, int BITS>
+__device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
+                                           int64_t c1, int G, const float (*qrot)[D], uint8_t *stages,
+                                           uint64_t *bars, float *mw, float *lw, float *accw) {
+  using S = Stage<FAM, BITS>;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const bool hv = g < G;
+  constexpr float CSC = (float)(1 << (BITS)) / 256.0f;  // 2^(b-8): undoes the code's byte position
+  constexpr float HALF_RANGE = (float)(1 << (BITS - 1));
+
+  float acc[32], accp[32];  // index blk*8 + u*2 + e <-> channel 32 blk + 8 tq + 4 e + u
+#pragma unroll
+  for (int i = 0; i < 32; ++i) acc[i] = accp[i] = 0.f;
+  float aoff[4] = {0.f, 0.f, 0.f, 0.f};
+  float m_run = -INFINITY, l_run = 0.f;
+  uint32_t qa[4][4];
+  float sigp = 0.f, qs[4] = {0.f, 0.f, 0.f, 0.f};
+  int64_t cur_page = -1;
+  bool ok = true;
+
+  const int nj = (int)(c1 - c0);
+  if (lane == 0) {
+    for (int j = 0; j < S::NST && j < nj; ++j)
+      issue_chunk<FAM, BITS>(L, seq, head, a + (c0 + j) * CH, stages + j * S::BYTES, &bars[j]);
+  }
+  for (int j = 0; j < nj && ok; ++j) {
+    const int si = j % S::NST;
+    uint8_t *st = stages + si * S::BYTES;
+    if (!mbar_wait(&bars[si], (uint32_t)((j / S::NST) & 1), L.status)) {
+      ok = false;
+      break;
+    }
+    const int64_t i0 = a + (c0 + j) * CH;
+    const int64_t page = i0 / GROUP;
+    const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
+    if (page != cur_page && (FAM == FAM_KVARN || cur_page < 0)) {
+      // query of head g in 16-bit fixed point (two int8 limbs), times the page's K channel
+      // scales c for kvarn; the lane covers channels 32 blk + 8 tq + (0..7)
+      float qv[32], amax = 0.f;
+      const __half *ck = reinterpret_cast<const __half *>(st + S::KCS);
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int ch = 32 * blk + 8 * tq + i;
+          float v = hv ? qrot[g][ch] : 0.f;
+          if (FAM == FAM_KVARN) v *= h2f(ck, ch);
+          qv[blk * 8 + i] = v;
+          amax = fmaxf(amax, fabsf(v));
+        }
+      amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+      const float inv = amax > 0.f ? QFIX / amax : 0.f;
+      sigp = amax / QFIX * CSC;
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        int hi[8], lo[8];
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int qi = __float2int_rn(qv[blk * 8 + i] * inv);
+          hi[i] = (qi + 128) >> 8;
+          lo[i] = qi - (hi[i] << 8);
+          sum += qv[blk * 8 + i];
+        }
+        qa[blk][0] = pack_s8(hi[0], hi[1], hi[2], hi[3]);
+        qa[blk][1] = pack_s8(lo[0], lo[1], lo[2], lo[3]);
+        qa[blk][2] = pack_s8(hi[4], hi[5], hi[6], hi[7]);
+        qa[blk][3] = pack_s8(lo[4], lo[5], lo[6], lo[7]);
+        if (FAM == FAM_ASYM) {
+          sum += __shfl_xor_sync(FULL, sum, 1);
+          sum += __shfl_xor_sync(FULL, sum, 2);
+          qs[blk] = sum;
+        }
+      }
+    }
+    cur_page = page;
+
+    const __half *dk = reinterpret_cast<const __half *>(st + S::KD);
+    const __half *dvv = reinterpret_cast<const __half *>(st + S::VD);
+    const __half *mk = reinterpret_cast<const __half *>(st + S::KM);
+    const __half *mvv = reinterpret_cast<const __half *>(st + S::VM);
+    const __half *tk = reinterpret_cast<const __half *>(st + S::KT);
+    const __half *tvv = reinterpret_cast<const __half *>(st + S::VT);
+
+    // ---- Q.K: n-tile r, column n holds token 16(r>>1) + 4(n>>1) + 2(r&1) + (n&1), so that
+    //      the lane ends with the scores of tokens 4tq+(0..3) and 16+4tq+(0..3)
+    float sc[8];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      KTok<FAM, BITS> kt;
+      kt.load(st + S::KC + (16 * (r >> 1) + 4 * (g >> 1) + 2 * (r & 1) + (g & 1)) * 16 * BITS, tq);
+      float x0 = 0.f, x1 = 0.f, o0 = 0.f, o1 = 0.f;
+      const int t0 = 16 * (r >> 1) + 4 * tq + 2 * (r & 1);
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        uint32_t b0, b1;
+        kt.frag(blk, tq, b0, b1);
+        int c[4] = {0, 0, 0, 0};
+        mma_s8(c, qa[blk], b0, b1);
+        const float d0 = h2f(dk, t0 * 4 + blk), d1 = h2f(dk, (t0 + 1) * 4 + blk);
+        x0 = fmaf(d0, (float)(c[0] * 256 + c[2]), x0);
+        x1 = fmaf(d1, (float)(c[1] * 256 + c[3]), x1);
+        if (FAM == FAM_ASYM) {
+          o0 = fmaf(fmaf(d0, HALF_RANGE, h2f(mk, t0 * 4 + blk)), qs[blk], o0);
+          o1 = fmaf(fmaf(d1, HALF_RANGE, h2f(mk, (t0 + 1) * 4 + blk)), qs[blk], o1);
+        }
+      }
+      float s0 = x0 * sigp + o0, s1 = x1 * sigp + o1;
+      if (FAM == FAM_KVARN) {
+        s0 *= h2f(tk, t0);
+        s1 *= h2f(tk, t0 + 1);
+      }
+      sc[2 * r] = t0 < nvalid ? s0 : -INFINITY;
+      sc[2 * r + 1] = t0 + 1 < nvalid ? s1 : -INFINITY;
+    }
+
+    // ---- online softmax (head g; the 4 lanes of a group hold the chunk's 32 tokens)
+    float cmax = sc[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) cmax = fmaxf(cmax, sc[k]);
+    cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 1));
+    cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 2));
+    const float mn = fmaxf(m_run, cmax);
+    const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mn);
+    float p[8], psum = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      p[k] = sc[k] == -INFINITY ? 0.f : exp2f(sc[k] - mn);
+      psum += p[k];
+    }
+    if (alpha != 1.f) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        acc[i] *= alpha;
+        accp[i] *= alpha;
+      }
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) aoff[blk] *= alpha;
+    }
+    l_run = l_run * alpha + psum;
+    m_run = mn;
+
+    // ---- P.V: weights w = p * t * d per (token, block) in 16-bit fixed point, scaled per
+    //      block by the chunk's largest t*d (p <= 1); rows past the end of the context may
+    //      hold stale bytes and are kept out of every sum
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      float td[8], tdm = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int tok = 16 * (k >> 2) + 4 * tq + (k & 3);
+        const bool vk = tok < nvalid;
+        float v = h2f(dvv, tok * 4 + blk);
+        if (FAM == FAM_KVARN) v *= h2f(tvv, tok);
+        v = vk ? v : 0.f;
+        td[k] = v;
+        tdm = fmaxf(tdm, v);
+        if (FAM == FAM_ASYM) {
+          const float mv = vk ? h2f(mvv, tok * 4 + blk) : 0.f;
+          aoff[blk] = fmaf(p[k], fmaf(v, HALF_RANGE, mv), aoff[blk]);
+        }
+      }
+      tdm = fmaxf(tdm, __shfl_xor_sync(FULL, tdm, 1));
+      tdm = fmaxf(tdm, __shfl_xor_sync(FULL, tdm, 2));
+      const float inv = tdm > 0.f ? QFIX / tdm : 0.f;
+      uint32_t wb[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) wb[k] = __float_as_uint(fmaf(p[k], td[k] * inv, MAGIC));
+      uint32_t wa[4];
+      {
+        const uint32_t x = __byte_perm(wb[0], wb[1], 0x5140), y = __byte_perm(wb[2], wb[3], 0x5140);
+        wa[0] = __byte_perm(x, y, 0x7632);
+        wa[1] = __byte_perm(x, y, 0x5410) ^ 0x80808080u;
+      }
+      {
+        const uint32_t x = __byte_perm(wb[4], wb[5], 0x5140), y = __byte_perm(wb[6], wb[7], 0x5140);
+        wa[2] = __byte_perm(x, y, 0x7632);
+        wa[3] = __byte_perm(x, y, 0x5410) ^ 0x80808080u;
+      }
+      VQuad<FAM, BITS> v0, v1;
+      v0.load(st + S::VC + tq * S::QS, blk, g);
+      v1.load(st + S::VC + (4 + tq) * S::QS, blk, g);
+      const float scl = tdm / QFIX * CSC;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        int c[4] = {0, 0, 0, 0};
+        mma_s8(c, wa, v0.frag(u, g), v1.frag(u, g));
+        float *dst = FAM == FAM_KVARN ? accp : acc;
+        dst[blk * 8 + u * 2 + 0] = fmaf(scl, (float)(c[0] * 256 + c[2]), dst[blk * 8 + u * 2 + 0]);
+        dst[blk * 8 + u * 2 + 1] = fmaf(scl, (float)(c[1] * 256 + c[3]), dst[blk * 8 + u * 2 + 1]);
+      }
+    }
+
+    // kvarn: at the last chunk of a page fold the page's V channel scales c into acc
+    if (FAM == FAM_KVARN && (j + 1 == nj || (a + (c0 + j + 1) * CH) / GROUP != page)) {
+      const __half *cv = reinterpret_cast<const __half *>(st + S::VCS);
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int idx = blk * 8 + u * 2 + e;
+            acc[idx] = fmaf(h2f(cv, 32 * blk + 8 * tq + 4 * e + u), accp[idx], acc[idx]);
+            accp[idx] = 0.f;
+          }
+    }
+
+    __syncwarp();
+    if (lane == 0 && j + S::NST < nj) {
+      fence_proxy_async();  // this warp's reads of the stage come before the copy into it
+      issue_chunk<FAM, BITS>(L, seq, head, a + (c0 + j + S::NST) * CH, st, &bars[si]);
+    }
+  }
+  if (!ok) {
+    // drain: wait (bounded) for every copy still in flight before the stage memory is reused
+    for (int j = 0; j < nj && j < S::NST; ++j) mbar_wait(&bars[j], 0u, L.status);
+  }
+  l_run += __shfl_xor_sync(FULL, l_run, 1);
+  l_run += __shfl_xor_sync(FULL, l_run, 2);
+  if (FAM == FAM_ASYM) {
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      aoff[blk] += __shfl_xor_sync(FULL, aoff[blk], 1);
+      aoff[blk] += __shfl_xor_sync(FULL, aoff[blk], 2);
+    }
+  }
+  __syncwarp();
+  if (hv) {
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          accw[g * D + 32 * blk + 8 * tq + 4 * e + u] = acc[blk * 8 + u * 2 + e] + aoff[blk];
+    if (tq == 0) {
+      mw[g] = m_run;
+      lw[g] = l_run;
+    }
+  }
+}
+
+// Exact BF16 rows (the tail, or a whole BF16 cache) on CUDA cores: Q.K with one token per
+// lane, P.V with four channels per lane.  Tokens [c0*32 + a, ...) of this warp.
+__device__ __forceinline__ void warp_bf16(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
+                                          int64_t c1, int G, const float (*qraw)[D], float (*pst)[MAX_G],
+                                          float *mw, float *lw, float *accw) {
+  const int lane = threadIdx.x & 31;
+  float m[MAX_G], l[MAX_G], acc[MAX_G][4];
+#pragma unroll
+  for (int g = 0; g < MAX_G; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[g][e] = 0.f;
+  }
+  const __nv_bfloat16 *kbase = ring_row(L, seq, head, 0, 0);
+  const __nv_bfloat16 *vbase = ring_row(L, seq, head, 1, 0);
+  for (int64_t ci = c0; ci < c1; ++ci) {
+    const int64_t i0 = a + ci * CH;
+    const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
+    const bool valid = lane < nvalid;
+    const int64_t slot0 = i0 % L.ring_cap;  // ring row of token i0; later rows wrap
+    float sc[MAX_G];
+#pragma unroll
+    for (int g = 0; g < MAX_G; ++g) sc[g] = 0.f;
+    if (valid) {
+      int64_t sl = slot0 + lane;
+      if (sl >= L.ring_cap) sl -= L.ring_cap;
+      const uint4 *row = reinterpret_cast<const uint4 *>(kbase + sl * D);
+      uint4 raw[D / 8];
+#pragma unroll
+      for (int j8 = 0; j8 < D / 8; ++j8) raw[j8] = row[j8];
+#pragma unroll
+      for (int j8 = 0; j8 < D / 8; ++j8) {
+        float x[8];
+        const uint32_t w[4] = {raw[j8].x, raw[j8].y, raw[j8].z, raw[j8].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          x[2 * u] = __uint_as_float(w[u] << 16);
+          x[2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
+        }
+#pragma unroll
+        for (int g = 0; g < MAX_G; ++g) {
+          if (g >= G) break;
+          const float4 qa = *reinterpret_cast<const float4 *>(&qraw[g][8 * j8]);
+          const float4 qb = *reinterpret_cast<const float4 *>(&qraw[g][8 * j8 + 4]);
+          float t = sc[g];
+          t = fmaf(x[0], qa.x, t);
+          t = fmaf(x[1], qa.y, t);
+          t = fmaf(x[2], qa.z, t);
+          t = fmaf(x[3], qa.w, t);
+          t = fmaf(x[4], qb.x, t);
+          t = fmaf(x[5], qb.y, t);
+          t = fmaf(x[6], qb.z, t);
+          t = fmaf(x[7], qb.w, t);
+          sc[g] = t;
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < MAX_G; ++g) {
+      if (g >= G) break;
+      const float sv_ = valid ? sc[g] : -INFINITY;
+      const float mn = fmaxf(m[g], warp_max(sv_));
+      const float alpha = m[g] == -INFINITY ? 0.f : exp2f(m[g] - mn);
+      const float p = valid ? exp2f(sv_ - mn) : 0.f;
+      l[g] = l[g] * alpha + warp_sum(p);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[g][e] *= alpha;
+      m[g] = mn;
+      pst[lane][g] = p;
+    }
+    __syncwarp();
+    uint2 vr[CH];
+#pragma unroll
+    for (int t = 0; t < CH; ++t) {
+      int64_t sl = slot0 + t;
+      if (sl >= L.ring_cap) sl -= L.ring_cap;
+      vr[t] = t < nvalid ? reinterpret_cast<const uint2 *>(vbase + sl * D)[lane] : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int t = 0; t < CH; ++t) {
+      const float v0 = __uint_as_float(vr[t].x << 16), v1 = __uint_as_float(vr[t].x & 0xffff0000u);
+      const float v2 = __uint_as_float(vr[t].y << 16), v3 = __uint_as_float(vr[t].y & 0xffff0000u);
+      const float4 pa = *reinterpret_cast<const float4 *>(&pst[t][0]);
+      const float4 pb = *reinterpret_cast<const float4 *>(&pst[t][4]);
+      const float pp[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+      for (int g = 0; g < MAX_G; ++g) {
+        if (g >= G) break;
+        acc[g][0] = fmaf(pp[g], v0, acc[g][0]);
+        acc[g][1] = fmaf(pp[g], v1, acc[g][1]);
+        acc[g][2] = fmaf(pp[g], v2, acc[g][2]);
+        acc[g][3] = fmaf(pp[g], v3, acc[g][3]);
+      }
+    }
+    __syncwarp();
+  }
+#pragma unroll
+  for (int g = 0; g < MAX_G; ++g) {
+    if (g >= G) break;
+    if (lane == 0) {
+      mw[g] = m[g];
+      lw[g] = l[g];
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) accw[g * D + 4 * lane + e] = acc[g][e];
+  }
+}
+
+// Shared memory of the kernel (dynamic): fixed part + per-warp stage area (also used for the
+// warps' accumulators once the chunks are done).
+struct SmemFixed {
+  float qraw[MAX_G][D];
+  float qrot[MAX_G][D];
+  float pst[NW][CH][MAX_G];
+  float mw[NW][MAX_G], lw[NW][MAX_G];
+  float fw[MAXSPL][MAX_G];   // merge: weight of each split
+  float fl[MAXSPL][MAX_G];   // merge: l of each split
+  float red[MAX_G][D];       // merge: second half of the split sum
+  float Ls[MAX_G];
+  uint64_t bars[NW][4];
+  int is_last;
+};
+
+template <int FAM, int BITS>
+__host__ __device__ constexpr int warp_area() {
+  if constexpr (FAM == FAM_BF16) {
+    return MAX_G * D * 4;
+  } else {
+    constexpr int s = Stage<FAM, BITS>::NST * Stage<FAM, BITS>::BYTES;
+    return s > MAX_G * D * 4 ? s : MAX_G * D * 4;
+  }
 }
 
 template <int FAM, int BITS>
-__global__ void __launch_bounds__(DT) k_decode(LayerView L, DArgs A) {
-  __shared__ float qraw[MAX_G][D];
-  __shared__ float qrot[MAX_G][D];
-  __shared__ float qc[NW][MAX_G][D];
-  __shared__ float ps[NW][MAX_G][CH];
-  __shared__ float qsum[MAX_G][4];
-  __shared__ float mw[NW][MAX_G], lw[NW][MAX_G];
-  __shared__ float accw[NW][MAX_G][D];
-  __shared__ int is_last;
+__host__ __device__ constexpr size_t smem_bytes() {
+  return ((sizeof(SmemFixed) + 127) / 128) * 128 + (size_t)NW * warp_area<FAM, BITS>();
+}
+
+template <int FAM, int BITS>
+__global__ void __launch_bounds__(DT, 1) k_decode(LayerView L, DArgs A) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  SmemFixed &F = *reinterpret_cast<SmemFixed *>(smem);
+  uint8_t *warp_mem = smem + ((sizeof(SmemFixed) + 127) / 128) * 128;
+  constexpr int WA = warp_area<FAM, BITS>();
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bid = blockIdx.x;
@@ -101,6 +683,7 @@ __global__ void __launch_bounds__(DT) k_decode(LayerView L, DArgs A) {
   const int G = A.G;
   const bool tail = sp >= s.nsq;
   int64_t a, b;
+  int64_t nch;
   if (!tail) {
     a = (int64_t)sp * s.cps_q * CH;
     b = min(a + (int64_t)s.cps_q * CH, s.Q);
@@ -108,11 +691,23 @@ __global__ void __launch_bounds__(DT) k_decode(LayerView L, DArgs A) {
     a = s.Q + (int64_t)(sp - s.nsq) * s.cps_t * CH;
     b = min(a + (int64_t)s.cps_t * CH, s.n);
   }
+  nch = b > a ? (b - a + CH - 1) / CH : 0;
+  // contiguous chunk range of this warp
+  const int64_t per = (nch + NW - 1) / NW;
+  const int64_t c0 = min((int64_t)warp * per, nch), c1 = min(c0 + per, nch);
 
-  // query rows of this KV head, pre-scaled by softmax_scale * log2(e)
-  for (int idx = tid; idx < G * D; idx += DT) {
+  if (lane == 0 && FAM != FAM_BF16 && !tail) {
+    for (int j = 0; j < 4; ++j) mbar_init(&F.bars[warp][j], 1);
+    fence_proxy_async();
+  }
+  // query rows of this KV head, pre-scaled by softmax_scale * log2(e); heads >= G are 0
+  for (int idx = tid; idx < MAX_G * D; idx += DT) {
     const int g = idx / D, j = idx % D;
-    qraw[g][j] = A.q[((int64_t)s.row * A.hkv * G + head * G + g) * D + j] * A.qscale;
+    F.qraw[g][j] = g < G ? A.q[((int64_t)s.row * A.hkv * G + head * G + g) * D + j] * A.qscale : 0.f;
+  }
+  for (int idx = tid; idx < NW * MAX_G; idx += DT) {
+    F.mw[idx / MAX_G][idx % MAX_G] = -INFINITY;
+    F.lw[idx / MAX_G][idx % MAX_G] = 0.f;
   }
   __syncthreads();
   if (!tail && A.rotk) {
@@ -120,7 +715,7 @@ __global__ void __launch_bounds__(DT) k_decode(LayerView L, DArgs A) {
     if (tid < G) {
       float r[D];
 #pragma unroll
-      for (int j = 0; j < D; ++j) r[j] = qraw[tid][j];
+      for (int j = 0; j < D; ++j) r[j] = F.qraw[tid][j];
 #pragma unroll
       for (int h = 1; h < D; h <<= 1) {
 #pragma unroll
@@ -132,253 +727,137 @@ __global__ void __launch_bounds__(DT) k_decode(LayerView L, DArgs A) {
         }
       }
 #pragma unroll
-      for (int j = 0; j < D; ++j) qrot[tid][j] = r[j] * kKappa();
+      for (int j = 0; j < D; ++j) F.qrot[tid][j] = r[j] * kKappa();
     }
   } else {
-    for (int idx = tid; idx < G * D; idx += DT) qrot[idx / D][idx % D] = qraw[idx / D][idx % D];
-  }
-  __syncthreads();
-  if (FAM == FAM_ASYM && tid < G * 4) {
-    const int g = tid / 4, bb = tid % 4;
-    float sum = 0.f;
-    for (int e = 0; e < 32; ++e) sum += qrot[g][32 * bb + e];
-    qsum[g][bb] = sum;
+    for (int idx = tid; idx < MAX_G * D; idx += DT) F.qrot[idx / D][idx % D] = F.qraw[idx / D][idx % D];
   }
   __syncthreads();
 
-  float m[MAX_G], l[MAX_G], acc[MAX_G][4];
-#pragma unroll
-  for (int g = 0; g < MAX_G; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
-#pragma unroll
-    for (int bb = 0; bb < 4; ++bb) acc[g][bb] = 0.f;
-  }
-
-  const int64_t nch = (b - a + CH - 1) / CH;
-  int64_t cur_page = -1;
-  float cv[4] = {1.f, 1.f, 1.f, 1.f};  // V channel scales of the current page (kvarn)
-  for (int64_t ci = warp; ci < nch; ci += NW) {
-    const int64_t i0 = a + ci * CH;
-    const int64_t i = i0 + lane;
-    const bool valid = i < b;
-    float sc[MAX_G];
-#pragma unroll
-    for (int g = 0; g < MAX_G; ++g) sc[g] = 0.f;
-    const uint8_t *sk = nullptr, *sv = nullptr;
-    const SubLayout lay = sub_layout(FAM, BITS);
-    if constexpr (FAM != FAM_BF16) {
-      if (!tail) {
-        const int64_t page = i0 / GROUP;
-        sk = subpage_ptr(L, s.seq, page, head, 0);
-        sv = subpage_ptr(L, s.seq, page, head, 1);
-        const float *qq = &qrot[0][0];
-        if (FAM == FAM_KVARN) {
-          if (page != cur_page) {
-            const __half *ck = reinterpret_cast<const __half *>(sk + lay.c);
-            const __half *cvh = reinterpret_cast<const __half *>(sv + lay.c);
-            for (int idx = lane; idx < G * D; idx += 32)
-              qc[warp][idx / D][idx % D] = qrot[idx / D][idx % D] * __half2float(ck[idx % D]);
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) cv[bb] = __half2float(cvh[lane + 32 * bb]);
-            __syncwarp();
-            cur_page = page;
-          }
-          qq = &qc[warp][0][0];
-        }
-        if (valid) {
-          const int tip = (int)(i % GROUP);
-          uint32_t w[4 * BITS];
-          const uint4 *src = reinterpret_cast<const uint4 *>(sk + tip * 16 * BITS);
-#pragma unroll
-          for (int k = 0; k < BITS; ++k) reinterpret_cast<uint4 *>(w)[k] = src[k];
-          const __half *dk = reinterpret_cast<const __half *>(sk + lay.d);
-#pragma unroll
-          for (int blk = 0; blk < 4; ++blk) {
-            float ab[MAX_G];
-#pragma unroll
-            for (int g = 0; g < MAX_G; ++g) ab[g] = 0.f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int ch = 32 * blk + e;
-              const float cval = (float)code_value<FAM, BITS>(k_field_w<BITS>(w, ch));
-#pragma unroll
-              for (int g = 0; g < MAX_G; ++g)
-                if (g < G) ab[g] = fmaf(cval, qq[g * D + ch], ab[g]);
-            }
-            const float d = __half2float(dk[tip * 4 + blk]);
-            float mk = 0.f;
-            if (FAM == FAM_ASYM) mk = __half2float(reinterpret_cast<const __half *>(sk + lay.m)[tip * 4 + blk]);
-#pragma unroll
-            for (int g = 0; g < MAX_G; ++g) {
-              sc[g] = fmaf(d, ab[g], sc[g]);
-              if (FAM == FAM_ASYM) sc[g] = fmaf(mk, qsum[g][blk], sc[g]);
-            }
-          }
-          if (FAM == FAM_KVARN) {
-            const float t = __half2float(reinterpret_cast<const __half *>(sk + lay.t)[tip]);
-#pragma unroll
-            for (int g = 0; g < MAX_G; ++g) sc[g] *= t;
-          }
-        }
-      }
+  float *accw = reinterpret_cast<float *>(warp_mem + (size_t)warp * WA);  // [MAX_G][D] after the chunks
+  if constexpr (FAM != FAM_BF16) {
+    if (!tail) {
+      warp_quant<FAM, BITS>(L, s.seq, head, a, b, c0, c1, G, F.qrot, warp_mem + (size_t)warp * WA, F.bars[warp],
+                            F.mw[warp], F.lw[warp], accw);
+    } else {
+      for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
+      __syncwarp();
+      warp_bf16(L, s.seq, head, a, b, c0, c1, G, F.qraw, F.pst[warp], F.mw[warp], F.lw[warp], accw);
     }
-    if (tail && valid) {
-      const __nv_bfloat16 *row = ring_row(L, s.seq, head, 0, i);
-      for (int j = 0; j < D; j += 8) {
-        uint4 raw = *reinterpret_cast<const uint4 *>(row + j);
-        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float x0 = __low2float(h2[u]), x1 = __high2float(h2[u]);
-#pragma unroll
-          for (int g = 0; g < MAX_G; ++g)
-            if (g < G) sc[g] = fmaf(x1, qraw[g][j + 2 * u + 1], fmaf(x0, qraw[g][j + 2 * u], sc[g]));
-        }
-      }
-    }
-    // online softmax over the chunk
-#pragma unroll
-    for (int g = 0; g < MAX_G; ++g) {
-      if (g >= G) break;
-      const float sv_ = valid ? sc[g] : -INFINITY;
-      const float cm = warp_max(sv_);
-      const float mn = fmaxf(m[g], cm);
-      const float alpha = m[g] == -INFINITY ? 0.f : exp2f(m[g] - mn);
-      const float p = valid ? exp2f(sv_ - mn) : 0.f;
-      l[g] = l[g] * alpha + warp_sum(p);
-#pragma unroll
-      for (int bb = 0; bb < 4; ++bb) acc[g][bb] *= alpha;
-      m[g] = mn;
-      ps[warp][g][lane] = p;
-    }
+  } else {
+    for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
     __syncwarp();
-    const int cnt = (int)((b - i0) < CH ? (b - i0) : CH);
-    for (int t = 0; t < cnt; ++t) {
-      const int64_t it = i0 + t;
-      float vv[4];
-      if (tail || FAM == FAM_BF16) {
-        const __nv_bfloat16 *row = ring_row(L, s.seq, head, 1, it);
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) vv[bb] = __bfloat162float(row[lane + 32 * bb]);
-      } else {
-        if constexpr (FAM != FAM_BF16) {
-          const SubLayout lv = sub_layout(FAM, BITS);
-          const int tip = (int)(it % GROUP);
-          const uint8_t *quad = sv + (tip >> 2) * 64 * BITS;
-          const __half *dv = reinterpret_cast<const __half *>(sv + lv.d);
-          float tv = 1.f;
-          if (FAM == FAM_KVARN) tv = __half2float(reinterpret_cast<const __half *>(sv + lv.t)[tip]);
-#pragma unroll
-          for (int bb = 0; bb < 4; ++bb) {
-            const int ch = lane + 32 * bb;
-            float val = (float)code_value<FAM, BITS>(v_field<BITS>(quad, tip & 3, ch)) *
-                        __half2float(dv[tip * 4 + bb]);
-            if (FAM == FAM_ASYM) val += __half2float(reinterpret_cast<const __half *>(sv + lv.m)[tip * 4 + bb]);
-            if (FAM == FAM_KVARN) val *= tv * cv[bb];
-            vv[bb] = val;
-          }
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < MAX_G; ++g) {
-        if (g >= G) break;
-        const float p = ps[warp][g][t];
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) acc[g][bb] = fmaf(p, vv[bb], acc[g][bb]);
-      }
-    }
-    __syncwarp();
-  }
-
-  // combine the warps of this CTA
-#pragma unroll
-  for (int g = 0; g < MAX_G; ++g) {
-    if (g >= G) break;
-    if (lane == 0) {
-      mw[warp][g] = m[g];
-      lw[warp][g] = l[g];
-    }
-#pragma unroll
-    for (int bb = 0; bb < 4; ++bb) accw[warp][g][lane + 32 * bb] = acc[g][bb];
+    warp_bf16(L, s.seq, head, a, b, c0, c1, G, F.qraw, F.pst[warp], F.mw[warp], F.lw[warp], accw);
   }
   __syncthreads();
+
+  // combine the warps of this CTA into its partial (m, l, acc) per query head
   const int slot0 = s.part0 + head * nspl;
-  for (int g = 0; g < G; ++g) {
-    float M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[w][g]);
-    float av = 0.f, lv = 0.f;
-    if (M != -INFINITY) {
-      for (int w = 0; w < NW; ++w) {
-        if (mw[w][g] == -INFINITY) continue;
-        const float f = exp2f(mw[w][g] - M);
-        av += f * accw[w][g][tid];
-        lv += f * lw[w][g];
+  if (tid < D) {
+    for (int g = 0; g < G; ++g) {
+      float M = -INFINITY;
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, F.mw[w][g]);
+      float av = 0.f, lv = 0.f;
+      if (M != -INFINITY) {
+        for (int w = 0; w < NW; ++w) {
+          if (F.mw[w][g] == -INFINITY) continue;
+          const float f = exp2f(F.mw[w][g] - M);
+          av += f * reinterpret_cast<const float *>(warp_mem + (size_t)w * WA)[g * D + tid];
+          lv += f * F.lw[w][g];
+        }
       }
-    }
-    float *dst = A.ws + ((int64_t)(slot0 + sp) * G + g) * PSTRIDE;
-    dst[2 + tid] = av;
-    if (tid == 0) {
-      dst[0] = M;
-      dst[1] = lv;
+      float *dst = A.ws + ((int64_t)(slot0 + sp) * G + g) * PSTRIDE;
+      dst[2 + tid] = av;
+      if (tid == 0) {
+        dst[0] = M;
+        dst[1] = lv;
+      }
     }
   }
 
-  // the last CTA of this (sequence, KV head) merges all splits
+  // the last CTA of this (sequence, KV head) merges all splits (atomic ticket; no waiting)
   __threadfence();
   __syncthreads();
   if (tid == 0) {
     const unsigned prev = atomicAdd(&A.tickets[s.seq * A.hkv + head], 1u);
-    is_last = prev == (unsigned)(nspl - 1);
+    F.is_last = prev == (unsigned)(nspl - 1);
   }
   __syncthreads();
-  if (!is_last) return;
+  if (!F.is_last) return;
   __threadfence();
-  float *buf = &accw[0][0][0];
-  for (int g = 0; g < G; ++g) {
+  const float *part = A.ws + (int64_t)slot0 * G * PSTRIDE;
+  for (int idx = tid; idx < nspl * G; idx += DT) {
+    const float *src = part + (int64_t)idx * PSTRIDE;  // split idx / G, head idx % G
+    F.fw[idx / G][idx % G] = __ldcg(src);
+    F.fl[idx / G][idx % G] = __ldcg(src + 1);
+  }
+  __syncthreads();
+  if (tid < G) {
     float M = -INFINITY;
-    for (int k = 0; k < nspl; ++k) M = fmaxf(M, __ldcg(A.ws + ((int64_t)(slot0 + k) * G + g) * PSTRIDE));
-    float Ls = 0.f, ar = 0.f, ap = 0.f;
-    if (M != -INFINITY) {
-      for (int k = 0; k < nspl; ++k) {
-        const float *src = A.ws + ((int64_t)(slot0 + k) * G + g) * PSTRIDE;
-        const float mk = __ldcg(src);
-        if (mk == -INFINITY) continue;
-        const float f = exp2f(mk - M);
-        Ls += f * __ldcg(src + 1);
-        const float v = f * __ldcg(src + 2 + tid);
-        if (k < s.nsq) ar += v;
-        else ap += v;
-      }
+    for (int k = 0; k < nspl; ++k) M = fmaxf(M, F.fw[k][tid]);
+    float Ls = 0.f;
+    for (int k = 0; k < nspl; ++k) {
+      const float f = (M == -INFINITY || F.fw[k][tid] == -INFINITY) ? 0.f : exp2f(F.fw[k][tid] - M);
+      F.fw[k][tid] = f;
+      Ls += f * F.fl[k][tid];
     }
-    if (A.rotv) {
-      buf[tid] = ar;
-      __syncthreads();
-      for (int h = 1; h < D; h <<= 1) {
-        const bool lo = !(tid & h);
-        float x = 0.f, y = 0.f;
-        if (lo) {
-          x = buf[tid];
-          y = buf[tid + h];
-        }
-        __syncthreads();
-        if (lo) {
-          buf[tid] = x + y;
-          buf[tid + h] = x - y;
-        }
-        __syncthreads();
+    F.Ls[tid] = Ls;
+  }
+  __syncthreads();
+  // thread = (half, channel): half 0 sums the quantized splits (stored basis), half 1 the
+  // tail splits (original basis)
+  const int ch = tid & (D - 1), half = tid >> 7;
+  const int k0 = half == 0 ? 0 : s.nsq, k1 = half == 0 ? s.nsq : nspl;
+  float sum[MAX_G];
+#pragma unroll
+  for (int g = 0; g < MAX_G; ++g) sum[g] = 0.f;
+  for (int k = k0; k < k1; ++k) {
+#pragma unroll
+    for (int g = 0; g < MAX_G; ++g)
+      if (g < G) sum[g] = fmaf(F.fw[k][g], __ldcg(part + ((int64_t)k * G + g) * PSTRIDE + 2 + ch), sum[g]);
+  }
+  if (half == 0) {
+#pragma unroll
+    for (int g = 0; g < MAX_G; ++g)
+      if (g < G) F.qraw[g][ch] = sum[g];  // q rows are no longer needed
+  } else {
+#pragma unroll
+    for (int g = 0; g < MAX_G; ++g)
+      if (g < G) F.red[g][ch] = sum[g];
+  }
+  __syncthreads();
+  if (A.rotv) {
+    // inverse rotation of the quantized part of every head: H.acc.kappa
+    for (int h = 1; h < D; h <<= 1) {
+      for (int idx = tid; idx < G * D / 2; idx += DT) {
+        const int g = idx / (D / 2), pr = idx % (D / 2);
+        const int lo = (pr / h) * 2 * h + (pr % h);
+        const float x = F.qraw[g][lo], y = F.qraw[g][lo + h];
+        F.qraw[g][lo] = x + y;
+        F.qraw[g][lo + h] = x - y;
       }
-      ar = buf[tid] * kKappa();
       __syncthreads();
     }
-    A.out[((int64_t)s.row * A.hkv * G + head * G + g) * D + tid] = Ls > 0.f ? (ar + ap) / Ls : 0.f;
+  }
+  for (int idx = tid; idx < G * D; idx += DT) {
+    const int g = idx / D, c = idx % D;
+    const float rot = A.rotv ? F.qraw[g][c] * kKappa() : F.qraw[g][c];
+    A.out[((int64_t)s.row * A.hkv * G + head * G + g) * D + c] = F.Ls[g] > 0.f ? (rot + F.red[g][c]) / F.Ls[g] : 0.f;
   }
   if (tid == 0) A.tickets[s.seq * A.hkv + head] = 0u;
 }
 
 template <int FAM, int BITS>
 cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st) {
-  k_decode<FAM, BITS><<<A.ncta, DT, 0, st>>>(L, A);
+  constexpr size_t smem = smem_bytes<FAM, BITS>();
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(k_decode<FAM, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_decode<FAM, BITS><<<A.ncta, DT, smem, st>>>(L, A);
   return cudaGetLastError();
 }
 
@@ -404,13 +883,12 @@ size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads) {
 int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &seqs, int n_q_heads,
                   const float *q, float scale, float *out, void *ws, size_t ws_bytes, cudaStream_t st) {
   if (c->p.type_k != c->p.type_v) return KVQ_E_UNSUPPORTED;
+  (void)ws_bytes;
   const LayerView L = layer_view(c, layer);
   const int hkv = c->p.n_kv_heads, G = n_q_heads / hkv;
-  const double tb = (double)token_bytes(c->fam_k, c->bits_k) + token_bytes(c->fam_v, c->bits_v);
-  double total = 0.0;
-  for (const DecodeSeq &d : seqs) total += hkv * ((double)d.Q * tb + (double)(d.n - d.Q) * 4.0 * D);
-  const double target = 4.0 * c->num_sms;
-  (void)ws_bytes;
+  // bytes per token of a (K+V) head pair; BF16 rows weigh double (CUDA-core path)
+  const double tbq = (double)token_bytes(c->fam_k, c->bits_k) + token_bytes(c->fam_v, c->bits_v);
+  const double tbt = 2.0 * 4.0 * D;
   for (size_t base = 0; base < seqs.size(); base += MAXS) {
     const size_t cnt = std::min<size_t>(MAXS, seqs.size() - base);
     DArgs A{};
@@ -424,6 +902,42 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
     A.out = out;
     A.ws = static_cast<float *>(ws);
     A.tickets = reinterpret_cast<uint32_t *>(c->base + c->off_tickets);
+    // split plan: about one CTA per SM in total, shared out by weighted bytes; every
+    // (sequence, part) with tokens gets at least one split per KV head
+    double wsum = 0.0;
+    for (size_t i = 0; i < cnt; ++i) {
+      const DecodeSeq &d = seqs[base + i];
+      wsum += (double)d.Q * tbq + (double)(d.n - d.Q) * tbt;
+    }
+    const double per_head = (double)c->num_sms / hkv;
+    std::vector<int> nq(cnt), nt(cnt);
+    std::vector<double> rq(cnt), rt(cnt);
+    int used = 0;
+    for (size_t i = 0; i < cnt; ++i) {
+      const DecodeSeq &d = seqs[base + i];
+      const int64_t nchq = (d.Q + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
+      const double sq = wsum > 0 ? per_head * d.Q * tbq / wsum : 0.0;
+      const double st_ = wsum > 0 ? per_head * (d.n - d.Q) * tbt / wsum : 0.0;
+      nq[i] = nchq ? (int)std::min<int64_t>(std::max(1, std::min((int)sq, MAXSQ)), nchq) : 0;
+      nt[i] = ncht ? (int)std::min<int64_t>(std::max(1, std::min((int)st_, MAXST)), ncht) : 0;
+      rq[i] = nchq ? sq - nq[i] : -1.0;
+      rt[i] = ncht ? st_ - nt[i] : -1.0;
+      used += hkv * (nq[i] + nt[i]);
+    }
+    // hand the CTAs left by rounding down to the largest remainders
+    while (used + hkv <= c->num_sms) {
+      int best = -1;
+      bool best_t = false;
+      double br = 0.0;
+      for (size_t i = 0; i < cnt; ++i) {
+        const DecodeSeq &d = seqs[base + i];
+        if (rq[i] > br && nq[i] < MAXSQ && nq[i] < (d.Q + CH - 1) / CH) { br = rq[i]; best = (int)i; best_t = false; }
+        if (rt[i] > br && nt[i] < MAXST && nt[i] < (d.n - d.Q + CH - 1) / CH) { br = rt[i]; best = (int)i; best_t = true; }
+      }
+      if (best < 0) break;
+      if (best_t) { ++nt[best]; rt[best] -= 1.0; } else { ++nq[best]; rq[best] -= 1.0; }
+      used += hkv;
+    }
     int cta = 0, part = 0;
     for (size_t i = 0; i < cnt; ++i) {
       const DecodeSeq &d = seqs[base + i];
@@ -433,18 +947,10 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
       s.n = d.n;
       s.Q = d.Q;
       const int64_t nchq = (d.Q + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
-      auto want = [&](double bytes, int64_t nchunks, int cap) -> int {
-        if (nchunks <= 0) return 0;
-        int w = total > 0 ? (int)std::ceil(target * hkv * bytes / total / hkv) : 1;
-        w = std::max(1, std::min<int>(w, cap));
-        return (int)std::min<int64_t>(w, nchunks);
-      };
-      int wq = want((double)d.Q * tb, nchq, MAXSQ);
-      int wt = want((double)(d.n - d.Q) * 4.0 * D, ncht, MAXST);
-      s.cps_q = wq ? (int)((nchq + wq - 1) / wq) : 1;
-      s.nsq = wq ? (int)((nchq + s.cps_q - 1) / s.cps_q) : 0;
-      s.cps_t = wt ? (int)((ncht + wt - 1) / wt) : 1;
-      s.nst = wt ? (int)((ncht + s.cps_t - 1) / s.cps_t) : 0;
+      s.cps_q = nq[i] ? (int)((nchq + nq[i] - 1) / nq[i]) : 1;
+      s.nsq = nq[i] ? (int)((nchq + s.cps_q - 1) / s.cps_q) : 0;
+      s.cps_t = nt[i] ? (int)((ncht + nt[i] - 1) / nt[i]) : 1;
+      s.nst = nt[i] ? (int)((ncht + s.cps_t - 1) / s.cps_t) : 0;
       if (s.nsq + s.nst == 0) s.nst = 1;  // empty sequence: one empty split writes zeros
       s.cta0 = cta;
       s.part0 = part;
@@ -452,7 +958,7 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
       part += hkv * (s.nsq + s.nst);
     }
     A.ncta = cta;
-    // q / out rows are indexed by DecodeSeq::row, the workspace slots restart per launch
+    // q / out rows are indexed by DecodeSeq::row; the workspace slots restart per launch
     if (dispatch(c->fam_k, c->bits_k, L, A, st) != cudaSuccess) return KVQ_E_CUDA;
     note_launches(1);
   }
