@@ -119,6 +119,18 @@ __device__ __forceinline__ void pack_codes(const int (&code)[4], uint8_t *sub, i
   }
 }
 
+// rint(RN(y / d)) (IEEE quotient, then round half to even) without a division in the common
+// case.  q = RN(y * RN(1/d)) is within 2 ulp of RN(y / d); when q is more than 4 ulp away from
+// the nearest half-integer both round to the same integer, otherwise the exact quotient is
+// taken.  (4 ulp of q is bounded by max(|q|, 1) * 2^-20.)
+__device__ __forceinline__ float rint_quotient(float y, float d, float rd) {
+  const float q = __fmul_rn(y, rd);
+  const float r = rintf(q);
+  const float tol = fmaxf(fabsf(q), 1.0f) * 9.5367431640625e-07f;
+  if (fabsf(fabsf(__fsub_rn(q, r)) - 0.5f) <= tol) return rintf(__fdiv_rn(y, d));
+  return r;
+}
+
 // ---- block quantizers (one token-head per warp; lane holds channels 4*lane..+3) ------
 
 template <int BITS, int WHICH>
@@ -131,12 +143,13 @@ __device__ __forceinline__ void quant_sym(const float (&y)[4], uint8_t *sub, con
   a = fmaxf(a, __shfl_xor_sync(FULL, a, 1));
   const __half dh = sat_half(__fdiv_rn(a, (float)QMAX));
   const float df = __half2float(dh);
+  const float rd = df != 0.0f ? __frcp_rn(df) : 0.0f;
   int code[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     int q = 0;
     if (df != 0.0f) {
-      float r = rintf(__fdiv_rn(y[e], df));
+      float r = rint_quotient(y[e], df, rd);
       r = fminf(fmaxf(r, (float)QMIN), (float)QMAX);
       q = (int)r;
     }
@@ -204,163 +217,252 @@ __global__ void __launch_bounds__(256) k_spill_qb(LayerView L, Work W, const __n
 
 constexpr int KV_THREADS = 256;
 constexpr int XS = D + 1;  // padded row stride of the fp32 tile in shared memory
-constexpr size_t KVARN_SMEM =
-    sizeof(float) * ((size_t)GROUP * XS + GROUP /*u*/ + GROUP /*t*/ + D /*c*/ + D /*w*/ + 8 * GROUP /*part*/ +
-                     D /*rc*/ + GROUP /*rt*/);
 
-// One CTA (256 threads) per (kvarn group, head).  Per sequence, s.a is the first group
-// the append touches (it may be a partial group that grows) and s.b the quantized length
-// Q(n1) after the append; items enumerate (group, head).
-template <int BITS, int WHICH>
+struct KvarnSmem {
+  float X[GROUP * XS];  // rotated rows x (fp32), padded rows
+  float uS[32][8];      // 1/t^2 of token l + 32 k at [l][k]
+  float tS[GROUP];      // token scales t
+  float cS[D];          // channel scales c
+  float wS[D];          // 1/c^2
+  float part[8][GROUP]; // token-sum partials of the 8 channel runs
+  float rc[D];          // 1/fp16(c)
+  float rt[GROUP];      // 1/fp16(t)
+};
+
+// d = a*b + c on two fp32 lanes, each rounded once (the same result as two fmaf)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long ra, rb, rc, rd;
+  memcpy(&ra, &a, 8);
+  memcpy(&rb, &b, 8);
+  memcpy(&rc, &c, 8);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  float2 d;
+  memcpy(&d, &rd, 8);
+  return d;
+}
+
+// One CTA (256 threads) per (kvarn group, head, K or V).  Per sequence, s.a is the first
+// group the append touches (it may be a partial group that grows) and s.b the quantized
+// length Q(n1) after the append; items enumerate (which, group, head) with which = 0 for the
+// first W.total/2 items when K and V are processed by one launch (W.which == 2).
+template <int BITS>
 __global__ void __launch_bounds__(KV_THREADS, 1)
-    k_spill_kvarn(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in, int iters) {
-  extern __shared__ float sm[];
-  float *X = sm;
-  float *u = X + GROUP * XS;
-  float *tt = u + GROUP;
-  float *cj = tt + GROUP;
-  float *wj = cj + D;
-  float *part = wj + D;
-  float *rc = part + 8 * GROUP;
-  float *rt = rc + D;
+    k_spill_kvarn(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in_k, const __nv_bfloat16 *__restrict__ in_v,
+                  int iters) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  KvarnSmem &S = *reinterpret_cast<KvarnSmem *>(smem_raw);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t item = blockIdx.x;
+  int64_t item = blockIdx.x;
+  int which = W.which;
+  if (which == 2) {
+    const int64_t half = W.total / 2;
+    which = item >= half ? 1 : 0;
+    if (which) item -= half;
+  }
+  const __nv_bfloat16 *in = which ? in_v : in_k;
   const SeqWork &s = W.s[find_seq(W, item)];
   const int64_t local = item - s.item0;
   const int head = (int)(local % L.hkv);
   const int64_t g = s.a + local / L.hkv;
   const int64_t g0 = g * GROUP;
-  const int64_t Q1 = s.b;  // quantized length after the append
+  const int64_t Q1 = s.b;
   const int ng = (int)((Q1 - g0) < GROUP ? (Q1 - g0) : GROUP);
   const SubLayout lay = sub_layout(FAM_KVARN, BITS);
-  uint8_t *sub = subpage_ptr(L, s.seq, g, head, WHICH);
+  uint8_t *sub = subpage_ptr(L, s.seq, g, head, which);
 
-  // 1. load the group's BF16 rows (ring or new input) as fp32
-  for (int i = warp; i < ng; i += 8) {
-    float x[4];
-    load4(src_row(L, s, head, WHICH, g0 + i, in), lane, x);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) X[i * XS + 4 * lane + e] = x[e];
-  }
-  __syncthreads();
-
-  // 2. Walsh-Hadamard rotation of each row: stages h = 1..64 ascending, then times kappa
+  // 1. each thread rotates one row in registers: BF16 -> fp32, butterfly h = 1..64, x kappa
   if (tid < ng) {
+    const uint4 *row = reinterpret_cast<const uint4 *>(src_row(L, s, head, which, g0 + tid, in));
     float r[D];
 #pragma unroll
-    for (int j = 0; j < D; ++j) r[j] = X[tid * XS + j];
+    for (int j8 = 0; j8 < D / 8; ++j8) {
+      const uint4 raw = row[j8];
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        r[8 * j8 + 2 * u] = __uint_as_float(w[u] << 16);
+        r[8 * j8 + 2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
+      }
+    }
 #pragma unroll
     for (int h = 1; h < D; h <<= 1) {
 #pragma unroll
       for (int j = 0; j < D; ++j) {
         if (j & h) continue;
-        const float a = r[j], b = r[j + h];
-        r[j] = __fadd_rn(a, b);
-        r[j + h] = __fsub_rn(a, b);
+        const float x = r[j], y = r[j + h];
+        r[j] = __fadd_rn(x, y);
+        r[j + h] = __fsub_rn(x, y);
       }
     }
 #pragma unroll
-    for (int j = 0; j < D; ++j) X[tid * XS + j] = __fmul_rn(r[j], kKappa());
-    tt[tid] = 1.0f;
+    for (int j = 0; j < D; ++j) S.X[tid * XS + j] = __fmul_rn(r[j], kKappa());
   }
+  if (tid < GROUP) S.uS[tid & 31][tid >> 5] = 1.0f;  // first iteration: t = 1
   __syncthreads();
 
-  // 3. Sinkhorn, scale-only form.  Thread (warp w, lane l) covers channels 16w..16w+15 and
-  //    tokens l, l+32, ..., l+224: channel sums chain over its tokens then xor-butterfly
-  //    over lanes (16, 8, 4, 2, 1); token sums chain over its 16 channels, then the 8 warp
-  //    partials are combined by an xor butterfly (4, 2, 1).
+  // 2. Sinkhorn on the squared tile held in registers: thread (warp w, lane l) covers channels
+  //    16w..16w+15 and tokens l + 32k (k = 0..7); rows past the group end square to 0.
+  //    x2p[k/2][c] holds tokens (2(k/2), 2(k/2)+1) of channel c for the packed token sums.
+  float2 x2p[4][16];
+#pragma unroll
+  for (int kp = 0; kp < 4; ++kp)
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i0 = lane + 32 * (2 * kp), i1 = lane + 32 * (2 * kp + 1);
+      const float x0 = i0 < ng ? S.X[i0 * XS + 16 * warp + c] : 0.0f;
+      const float x1 = i1 < ng ? S.X[i1 * XS + 16 * warp + c] : 0.0f;
+      x2p[kp][c] = make_float2(__fmul_rn(x0, x0), __fmul_rn(x1, x1));
+    }
   const float fng = (float)ng;
+  // channel index this lane ends with after the recursive-halving reduction
+  const int cidx = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
   for (int it = 0; it < iters; ++it) {
-    if (tid < ng) u[tid] = __fdiv_rn(1.0f, __fmul_rn(tt[tid], tt[tid]));
-    __syncthreads();
-#pragma unroll 4
-    for (int cc = 0; cc < 16; ++cc) {
-      const int j = 16 * warp + cc;
+    // channel step: S_j = sum_i x2_ij u_i (chain over this lane's tokens, then the butterfly
+    // 16, 8, 4, 2, 1 across lanes done by recursive halving)
+    float u[8];
+    {
+      const float4 ua = *reinterpret_cast<const float4 *>(&S.uS[lane][0]);
+      const float4 ub = *reinterpret_cast<const float4 *>(&S.uS[lane][4]);
+      u[0] = ua.x; u[1] = ua.y; u[2] = ua.z; u[3] = ua.w;
+      u[4] = ub.x; u[5] = ub.y; u[6] = ub.z; u[7] = ub.w;
+    }
+    float v[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
       float acc = 0.0f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int i = lane + 32 * k;
-        if (i < ng) {
-          const float x = X[i * XS + j];
-          acc = __fmaf_rn(__fmul_rn(x, x), u[i], acc);
-        }
+      for (int kp = 0; kp < 4; ++kp) {
+        acc = __fmaf_rn(x2p[kp][c].x, u[2 * kp], acc);
+        acc = __fmaf_rn(x2p[kp][c].y, u[2 * kp + 1], acc);
       }
+      v[c] = acc;
+    }
+    {  // level 16: keep channels [8 b4, 8 b4 + 8)
+      const bool hi = lane & 16;
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL, acc, o));
-      if (lane == 0) {
-        const float c = acc > 0.0f ? __fsqrt_rn(__fdiv_rn(acc, fng)) : 1.0f;
-        cj[j] = c;
-        wj[j] = __fdiv_rn(1.0f, __fmul_rn(c, c));
+      for (int c = 0; c < 8; ++c) {
+        const float send = hi ? v[c] : v[c + 8];
+        const float keep = hi ? v[c + 8] : v[c];
+        v[c] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 16));
       }
     }
-    __syncthreads();
+    {  // level 8
+      const bool hi = lane & 8;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = lane + 32 * k;
-      if (i < ng) {
-        float acc = 0.0f;
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-          const int j = 16 * warp + cc;
-          const float x = X[i * XS + j];
-          acc = __fmaf_rn(__fmul_rn(x, x), wj[j], acc);
-        }
-        part[warp * GROUP + i] = acc;
+      for (int c = 0; c < 4; ++c) {
+        const float send = hi ? v[c] : v[c + 4];
+        const float keep = hi ? v[c + 4] : v[c];
+        v[c] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 8));
       }
+    }
+    {  // level 4
+      const bool hi = lane & 4;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float send = hi ? v[c] : v[c + 2];
+        const float keep = hi ? v[c + 2] : v[c];
+        v[c] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 4));
+      }
+    }
+    {  // level 2
+      const bool hi = lane & 2;
+      const float send = hi ? v[0] : v[1];
+      const float keep = hi ? v[1] : v[0];
+      v[0] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 2));
+    }
+    v[0] = __fadd_rn(v[0], __shfl_xor_sync(FULL, v[0], 1));  // level 1
+    if ((lane & 1) == 0) {
+      const float c = v[0] > 0.0f ? __fsqrt_rn(__fdiv_rn(v[0], fng)) : 1.0f;
+      S.cS[16 * warp + cidx] = c;
+      S.wS[16 * warp + cidx] = __fdiv_rn(1.0f, __fmul_rn(c, c));
+    }
+    __syncwarp();
+    // token step: R_i = sum_j x2_ij w_j over this warp's 16 channels (chain in channel order),
+    // two tokens per packed FMA
+    float w[16];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const float4 wv = *reinterpret_cast<const float4 *>(&S.wS[16 * warp + 4 * q4]);
+      w[4 * q4] = wv.x; w[4 * q4 + 1] = wv.y; w[4 * q4 + 2] = wv.z; w[4 * q4 + 3] = wv.w;
+    }
+    float2 racc[4];
+#pragma unroll
+    for (int kp = 0; kp < 4; ++kp) {
+      float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) acc = ffma2(x2p[kp][c], make_float2(w[c], w[c]), acc);
+      racc[kp] = acc;
+    }
+#pragma unroll
+    for (int kp = 0; kp < 4; ++kp) {
+      S.part[warp][lane + 32 * (2 * kp)] = racc[kp].x;
+      S.part[warp][lane + 32 * (2 * kp + 1)] = racc[kp].y;
     }
     __syncthreads();
     if (tid < ng) {
       float p[8];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) p[r] = part[r * GROUP + tid];
+      for (int r = 0; r < 8; ++r) p[r] = S.part[r][tid];
       const float a0 = __fadd_rn(p[0], p[4]), a1 = __fadd_rn(p[1], p[5]);
       const float a2 = __fadd_rn(p[2], p[6]), a3 = __fadd_rn(p[3], p[7]);
-      const float b0 = __fadd_rn(a0, a2), b1 = __fadd_rn(a1, a3);
-      const float R = __fadd_rn(b0, b1);
-      tt[tid] = R > 0.0f ? __fsqrt_rn(__fdiv_rn(R, 128.0f)) : 1.0f;
+      const float R = __fadd_rn(__fadd_rn(a0, a2), __fadd_rn(a1, a3));
+      const float t = R > 0.0f ? __fsqrt_rn(__fdiv_rn(R, 128.0f)) : 1.0f;
+      S.tS[tid] = t;
+      S.uS[tid & 31][tid >> 5] = __fdiv_rn(1.0f, __fmul_rn(t, t));
     }
     __syncthreads();
   }
 
-  // 4. fp16 scales; normalization uses the stored (fp16) values
+  // 3. fp16 scales; normalization uses the stored (fp16) values
   if (tid < D) {
-    const __half h = scale_to_half(cj[tid]);
+    const __half h = scale_to_half(S.cS[tid]);
     reinterpret_cast<__half *>(sub + lay.c)[tid] = h;
-    rc[tid] = __fdiv_rn(1.0f, __half2float(h));
+    S.rc[tid] = __fdiv_rn(1.0f, __half2float(h));
   }
   if (tid < ng) {
-    const __half h = scale_to_half(tt[tid]);
+    const __half h = scale_to_half(S.tS[tid]);
     reinterpret_cast<__half *>(sub + lay.t)[tid] = h;
-    rt[tid] = __fdiv_rn(1.0f, __half2float(h));
+    S.rt[tid] = __fdiv_rn(1.0f, __half2float(h));
   }
   __syncthreads();
 
-  // 5. y = (x * rc_j) * rt_i, symmetric b-bit blocks of 32, packed
+  // 4. y = (x * rc_j) * rt_i, symmetric b-bit blocks of 32, packed
+  const float4 rc4 = *reinterpret_cast<const float4 *>(&S.rc[4 * lane]);
+  const float rcl[4] = {rc4.x, rc4.y, rc4.z, rc4.w};
   for (int i = warp; i < ng; i += 8) {
     float y[4];
+    const float rti = S.rt[i];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = 4 * lane + e;
-      y[e] = __fmul_rn(__fmul_rn(X[i * XS + j], rc[j]), rt[i]);
-    }
-    quant_sym<BITS, WHICH>(y, sub, lay, i, lane);
+    for (int e = 0; e < 4; ++e) y[e] = __fmul_rn(__fmul_rn(S.X[i * XS + 4 * lane + e], rcl[e]), rti);
+    if (which == 0)
+      quant_sym<BITS, 0>(y, sub, lay, i, lane);
+    else
+      quant_sym<BITS, 1>(y, sub, lay, i, lane);
   }
 }
 
 // Copies new rows that stay 16-bit into the ring: range per sequence [a, n1), rows
 // enumerated as (token, head), 16 threads per 256-byte row.
-__global__ void __launch_bounds__(256) k_tail_write(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in) {
+__global__ void __launch_bounds__(256) k_tail_write(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in_k,
+                                                    const __nv_bfloat16 *__restrict__ in_v) {
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t item = t >> 4;
+  int64_t item = t >> 4;
   const int part = (int)(t & 15);
   if (item >= W.total) return;
+  int which = W.which;
+  if (which == 2) {  // K and V in one launch: the first half of the items is K
+    const int64_t half = W.total / 2;
+    which = item >= half ? 1 : 0;
+    if (which) item -= half;
+  }
+  const __nv_bfloat16 *in = which ? in_v : in_k;
   const SeqWork &s = W.s[find_seq(W, item)];
   const int64_t local = item - s.item0;
   const int head = (int)(local % L.hkv);
   const int64_t p = s.a + local / L.hkv;
   const uint4 *src = reinterpret_cast<const uint4 *>(in + ((s.in_off + (p - s.n0)) * L.hkv + head) * D);
-  uint4 *dst = reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, W.which, p));
+  uint4 *dst = reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, which, p));
   dst[part] = src[part];
 }
 
@@ -379,29 +481,29 @@ cudaError_t spill_qb(int fam, int bits, const LayerView &L, const Work &W, const
   return cudaErrorInvalidValue;
 }
 
-template <int BITS, int WHICH>
-cudaError_t launch_kvarn_t(const LayerView &L, const Work &W, const __nv_bfloat16 *in, int iters, cudaStream_t st) {
+template <int BITS>
+cudaError_t launch_kvarn_t(const LayerView &L, const Work &W, const __nv_bfloat16 *in_k, const __nv_bfloat16 *in_v,
+                           int iters, cudaStream_t st) {
   static bool attr_set = false;  // per template instance; the attribute is per function
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_spill_kvarn<BITS, WHICH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)KVARN_SMEM);
+    cudaError_t e = cudaFuncSetAttribute(k_spill_kvarn<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(KvarnSmem));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_spill_kvarn<BITS, WHICH><<<(unsigned)W.total, KV_THREADS, KVARN_SMEM, st>>>(L, W, in, iters);
+  k_spill_kvarn<BITS><<<(unsigned)W.total, KV_THREADS, sizeof(KvarnSmem), st>>>(L, W, in_k, in_v, iters);
   return cudaGetLastError();
 }
 
-template <int WHICH>
-cudaError_t spill_kvarn(int bits, const LayerView &L, const Work &W, const __nv_bfloat16 *in, int iters,
-                        cudaStream_t st) {
+cudaError_t spill_kvarn(int bits, const LayerView &L, const Work &W, const __nv_bfloat16 *in_k,
+                        const __nv_bfloat16 *in_v, int iters, cudaStream_t st) {
   switch (bits) {
-    case 2: return launch_kvarn_t<2, WHICH>(L, W, in, iters, st);
-    case 3: return launch_kvarn_t<3, WHICH>(L, W, in, iters, st);
-    case 4: return launch_kvarn_t<4, WHICH>(L, W, in, iters, st);
-    case 5: return launch_kvarn_t<5, WHICH>(L, W, in, iters, st);
-    case 6: return launch_kvarn_t<6, WHICH>(L, W, in, iters, st);
-    case 8: return launch_kvarn_t<8, WHICH>(L, W, in, iters, st);
+    case 2: return launch_kvarn_t<2>(L, W, in_k, in_v, iters, st);
+    case 3: return launch_kvarn_t<3>(L, W, in_k, in_v, iters, st);
+    case 4: return launch_kvarn_t<4>(L, W, in_k, in_v, iters, st);
+    case 5: return launch_kvarn_t<5>(L, W, in_k, in_v, iters, st);
+    case 6: return launch_kvarn_t<6>(L, W, in_k, in_v, iters, st);
+    case 8: return launch_kvarn_t<8>(L, W, in_k, in_v, iters, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -417,11 +519,13 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
 
   for (size_t base = 0; base < seqs.size(); base += MAXS) {
     const size_t cnt = std::min<size_t>(MAXS, seqs.size() - base);
-    // 1. spill quantization, K then V
+    // 1. spill quantization: K and V in one launch when they share a kvarn type
+    const bool fused = c->p.type_k == c->p.type_v && fam[0] == FAM_KVARN;
     for (int which = 0; which < 2; ++which) {
       if (fam[which] == FAM_BF16) continue;
+      if (fused && which == 1) continue;
       Work W{};
-      W.which = which;
+      W.which = fused ? 2 : which;
       int64_t total = 0;
       for (size_t i = 0; i < cnt; ++i) {
         const AppendSeq &a = seqs[base + i];
@@ -446,20 +550,22 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
         total += items;
         ++W.n;
       }
-      W.total = total;
+      W.total = fused ? 2 * total : total;
       if (total == 0) continue;
       cudaError_t e = fam[which] == FAM_KVARN
-                          ? (which == 0 ? spill_kvarn<0>(bits[which], L, W, in[which], c->p.sinkhorn_iters, st)
-                                        : spill_kvarn<1>(bits[which], L, W, in[which], c->p.sinkhorn_iters, st))
+                          ? spill_kvarn(bits[which], L, W, in[0], in[1], c->p.sinkhorn_iters, st)
                           : (which == 0 ? spill_qb<0>(fam[which], bits[which], L, W, in[which], st)
                                         : spill_qb<1>(fam[which], bits[which], L, W, in[which], st));
       if (e != cudaSuccess) return KVQ_E_CUDA;
       note_launches(1);
     }
-    // 2. ring write of the new rows that stay 16-bit
+    // 2. ring write of the new rows that stay 16-bit (K and V in one launch when their
+    //    types keep the same rows)
+    const bool same_keep = fam[0] == fam[1];
     for (int which = 0; which < 2; ++which) {
+      if (same_keep && which == 1) continue;
       Work W{};
-      W.which = which;
+      W.which = same_keep ? 2 : which;
       int64_t total = 0;
       for (size_t i = 0; i < cnt; ++i) {
         const AppendSeq &a = seqs[base + i];
@@ -476,10 +582,10 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
         total += (s.b - s.a) * hkv;
         ++W.n;
       }
-      W.total = total;
+      W.total = same_keep ? 2 * total : total;
       if (total == 0) continue;
-      const int64_t threads = total * 16;
-      k_tail_write<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(L, W, in[which]);
+      const int64_t threads = W.total * 16;
+      k_tail_write<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(L, W, in[0], in[1]);
       if (cudaGetLastError() != cudaSuccess) return KVQ_E_CUDA;
       note_launches(1);
     }

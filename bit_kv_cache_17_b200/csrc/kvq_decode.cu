@@ -23,8 +23,9 @@ namespace kvq {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int DT = 256;      // threads per CTA (one CTA per SM)
-constexpr int NW = DT / 32;  // warps per CTA
+// warps per CTA (one CTA per SM): 12 where the per-warp stages fit, 8 for 6/8-bit codes
+__host__ __device__ constexpr int nwarps(int fam, int bits) { return (fam != 0 && bits <= 5) ? 12 : 8; }
+constexpr int NWMAX = 12;
 constexpr int CH = 32;       // tokens per chunk (one per lane)
 constexpr int MAXSQ = 48;    // max splits over the quantized prefix per (seq, head)
 constexpr int MAXST = 16;    // max splits over the tail per (seq, head)
@@ -79,6 +80,16 @@ __device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint
       "{%0,%1,%2,%3};\n"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// d = a.b + (bias in every element): the accumulator input is one shared register, so no
+// per-MMA reinitialization is needed
+__device__ __forceinline__ void mma_s8_bias(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, int bias) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(bias));
 }
 
 // field s (width W) of each byte of `word`, moved to bits [P, P+W) of the same byte
@@ -186,52 +197,23 @@ __device__ __forceinline__ float h2f(const __half *p, int i) { return __half2flo
 constexpr float QFIX = 32639.0f;              // 16-bit fixed point: 256*127 + 127
 constexpr float MAGIC = 12582912.0f + 128.0f;  // 1.5*2^23 (+128 offset for the limb split)
 
-// ---- TMA bulk copies + mbarriers (one pipeline per warp) ---------------------------------
+// ---- staging (one pipeline per warp) ---------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// global -> shared bulk copy (TMA, no multicast) completing on an mbarrier; 16-byte aligned
-// addresses, size a multiple of 16
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
-constexpr uint32_t kWaitLimit = 1u << 24;  // try_wait rounds before a wait is declared stuck
-constexpr int32_t kStatusWaitTimeout = 1;   // device status bit: a pipeline wait gave up
-
-// Bounded wait for a phase of an mbarrier; on timeout records the status bit and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  atomicOr(status, kStatusWaitTimeout);
-  return false;
+// 16-byte global -> shared copy through L2 (no register staging), tracked by commit groups
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 // Shared-memory image of one 32-token chunk of a quantized page (both K and V), filled by
-// bulk copies: codes of K, codes of V one quad per row with a 32-byte pad (so that the
-// lanes of one P.V fragment load hit distinct banks), then the fp16 scales.
+// cp.async: codes of K, codes of V one quad per row with a 32-byte pad (so that the lanes
+// of one P.V fragment load hit distinct banks), then the fp16 scales.
 template <int FAM, int BITS>
 struct Stage {
   static constexpr int QS = 64 * BITS + 32;  // padded quad stride
@@ -246,37 +228,61 @@ struct Stage {
   static constexpr int KCS = VT + (FAM == FAM_KVARN ? 64 : 0);
   static constexpr int VCS = KCS + (FAM == FAM_KVARN ? 256 : 0);
   static constexpr int BYTES = VCS + (FAM == FAM_KVARN ? 256 : 0);
-  static constexpr uint32_t TX = BYTES - 8 * 32;  // bytes the copies deliver (no pads)
-  static constexpr int NST = BITS <= 3 ? 4 : (BITS <= 5 ? 3 : 2);  // stages per warp
+  static constexpr int NST = BITS <= 3 ? 3 : 2;  // stages per warp
 };
 
-// Issues the bulk copies of chunk [i0, i0+32) of page `page` into `st` (one lane).
+// Copies chunk [i0, i0+32) (K and V codes, fp16 scales, and for kvarn the page's channel
+// scales) into the stage `st`, 16 bytes per lane and instruction, as one commit group.
 template <int FAM, int BITS>
-__device__ __forceinline__ void issue_chunk(const LayerView &L, int seq, int head, int64_t i0, uint8_t *st,
-                                            uint64_t *bar) {
+__device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head, int64_t i0, uint8_t *st, int lane) {
   using S = Stage<FAM, BITS>;
   const SubLayout lay = sub_layout(FAM, BITS);
   const int64_t page = i0 / GROUP;
   const int tip0 = (int)(i0 % GROUP);
   const uint8_t *sk = subpage_ptr(L, seq, page, head, 0);
   const uint8_t *sv = subpage_ptr(L, seq, page, head, 1);
-  mbar_expect_tx(bar, S::TX);
-  bulk_g2s(st + S::KC, sk + tip0 * 16 * BITS, 512 * BITS, bar);
+  constexpr int KP = 32 * BITS;  // 16-byte pieces of K codes (and of V codes)
+  constexpr int QP = 4 * BITS;   // pieces per V quad
+  const uint8_t *kc = sk + tip0 * 16 * BITS;
+  const uint8_t *vc = sv + (tip0 / 4) * 64 * BITS;
 #pragma unroll
-  for (int q = 0; q < 8; ++q) bulk_g2s(st + S::VC + q * S::QS, sv + (tip0 / 4 + q) * 64 * BITS, 64 * BITS, bar);
-  bulk_g2s(st + S::KD, sk + lay.d + tip0 * 8, 256, bar);
-  bulk_g2s(st + S::VD, sv + lay.d + tip0 * 8, 256, bar);
-  if constexpr (FAM == FAM_ASYM) {
-    bulk_g2s(st + S::KM, sk + lay.m + tip0 * 8, 256, bar);
-    bulk_g2s(st + S::VM, sv + lay.m + tip0 * 8, 256, bar);
+  for (int p = lane; p < KP; p += 32) cp_async16(st + S::KC + 16 * p, kc + 16 * p);
+#pragma unroll
+  for (int p = lane; p < KP; p += 32) {
+    const int q = p / QP, o = p % QP;
+    cp_async16(st + S::VC + q * S::QS + 16 * o, vc + q * 64 * BITS + 16 * o);
   }
-  if constexpr (FAM == FAM_KVARN) {
-    bulk_g2s(st + S::KT, sk + lay.t + tip0 * 2, 64, bar);
-    bulk_g2s(st + S::VT, sv + lay.t + tip0 * 2, 64, bar);
-    bulk_g2s(st + S::KCS, sk + lay.c, 256, bar);
-    bulk_g2s(st + S::VCS, sv + lay.c, 256, bar);
+  // fp16 scales: 16 pieces of d for K and V, + m (qb_1), + t, c (kvarn)
+  if (lane < 16) {
+    cp_async16(st + S::KD + 16 * lane, sk + lay.d + tip0 * 8 + 16 * lane);
+    cp_async16(st + S::VD + 16 * lane, sv + lay.d + tip0 * 8 + 16 * lane);
+    if constexpr (FAM == FAM_ASYM) {
+      cp_async16(st + S::KM + 16 * lane, sk + lay.m + tip0 * 8 + 16 * lane);
+      cp_async16(st + S::VM + 16 * lane, sv + lay.m + tip0 * 8 + 16 * lane);
+    }
+    if constexpr (FAM == FAM_KVARN) {
+      cp_async16(st + S::KCS + 16 * lane, sk + lay.c + 16 * lane);
+      cp_async16(st + S::VCS + 16 * lane, sv + lay.c + 16 * lane);
+    }
+  } else if (FAM == FAM_KVARN && lane < 24) {
+    const int l = lane - 16;  // 4 pieces each of t for K and V
+    if (l < 4)
+      cp_async16(st + S::KT + 16 * l, sk + lay.t + tip0 * 2 + 16 * l);
+    else
+      cp_async16(st + S::VT + 16 * (l - 4), sv + lay.t + tip0 * 2 + 16 * (l - 4));
   }
 }
+
+// Per-warp scale tables of one chunk, built with one token per lane.
+struct ChunkTabs {
+  float k[CH][4];   // K: d * t (kvarn) or d, per token and block (0 past the context end)
+  float v[4][CH];   // V: t * d * QFIX / max over the chunk (per block) -> weights in fixed point
+  float km[CH][4];  // qb_1 K: m + d * 2^(b-1)
+  float vm[CH][4];  // qb_1 V: m + d * 2^(b-1)
+};
+
+constexpr int kBias = 0x4B400000;       // float bits of 1.5 * 2^23
+constexpr float kBiasF = 12582912.0f;  // an int32 accumulator started at kBias reads as kBiasF + sum
 
 // Q.K and P.V of one warp over its chunks [c0, c1) of a quantized split starting at token a
 // (chunks are consecutive, so pages change rarely).  Writes the warp's online-softmax state
@@ -284,36 +290,42 @@ __device__ __forceinline__ void issue_chunk(const LayerView &L, int seq, int hea
 template <int FAM, int BITS>
 __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
                                            int64_t c1, int G, const float (*qrot)[D], uint8_t *stages,
-                                           uint64_t *bars, float *mw, float *lw, float *accw) {
+                                           ChunkTabs &T, float *mw, float *lw, float *accw) {
   using S = Stage<FAM, BITS>;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   const bool hv = g < G;
   constexpr float CSC = (float)(1 << (BITS)) / 256.0f;  // 2^(b-8): undoes the code's byte position
   constexpr float HALF_RANGE = (float)(1 << (BITS - 1));
+  constexpr float SCL = CSC / QFIX;
 
-  float acc[32], accp[32];  // index blk*8 + u*2 + e <-> channel 32 blk + 8 tq + 4 e + u
+  float acc[32];  // index blk*8 + u*2 + e <-> channel 32 blk + 8 tq + 4 e + u
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = accp[i] = 0.f;
+  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
   float aoff[4] = {0.f, 0.f, 0.f, 0.f};
   float m_run = -INFINITY, l_run = 0.f;
   uint32_t qa[4][4];
   float sigp = 0.f, qs[4] = {0.f, 0.f, 0.f, 0.f};
   int64_t cur_page = -1;
-  bool ok = true;
 
   const int nj = (int)(c1 - c0);
-  if (lane == 0) {
-    for (int j = 0; j < S::NST && j < nj; ++j)
-      issue_chunk<FAM, BITS>(L, seq, head, a + (c0 + j) * CH, stages + j * S::BYTES, &bars[j]);
+  // prologue: NST - 1 chunks in flight (one commit group each, empty groups past the end)
+#pragma unroll
+  for (int j = 0; j < S::NST - 1; ++j) {
+    if (j < nj) copy_chunk<FAM, BITS>(L, seq, head, a + (c0 + j) * CH, stages + j * S::BYTES, lane);
+    cp_async_commit();
   }
-  for (int j = 0; j < nj && ok; ++j) {
+#pragma unroll 1
+  for (int j = 0; j < nj; ++j) {
     const int si = j % S::NST;
     uint8_t *st = stages + si * S::BYTES;
-    if (!mbar_wait(&bars[si], (uint32_t)((j / S::NST) & 1), L.status)) {
-      ok = false;
-      break;
+    {  // keep NST - 1 chunks in flight: issue chunk j + NST - 1 into the stage read last round
+      const int jn = j + S::NST - 1;
+      if (jn < nj) copy_chunk<FAM, BITS>(L, seq, head, a + (c0 + jn) * CH, stages + (jn % S::NST) * S::BYTES, lane);
+      cp_async_commit();
     }
+    cp_async_wait<S::NST - 1>();  // chunk j has landed (for this lane's copies)
+    __syncwarp();                 // ... and for every lane's
     const int64_t i0 = a + (c0 + j) * CH;
     const int64_t page = i0 / GROUP;
     const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
@@ -334,8 +346,8 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
         }
       amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
-      const float inv = amax > 0.f ? QFIX / amax : 0.f;
-      sigp = amax / QFIX * CSC;
+      const float inv = amax > 0.f ? QFIX * __frcp_rn(amax) : 0.f;
+      sigp = amax * SCL;
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
         int hi[8], lo[8];
@@ -360,12 +372,55 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     }
     cur_page = page;
 
-    const __half *dk = reinterpret_cast<const __half *>(st + S::KD);
-    const __half *dvv = reinterpret_cast<const __half *>(st + S::VD);
-    const __half *mk = reinterpret_cast<const __half *>(st + S::KM);
-    const __half *mvv = reinterpret_cast<const __half *>(st + S::VM);
-    const __half *tk = reinterpret_cast<const __half *>(st + S::KT);
-    const __half *tvv = reinterpret_cast<const __half *>(st + S::VT);
+    // ---- scale tables: lane = token of the chunk; rows past the end of the context may hold
+    //      stale bytes and get zero scales, so they never reach a sum
+    float scl[4];
+    {
+      const bool vl = lane < nvalid;
+      const uint2 dkr = *reinterpret_cast<const uint2 *>(st + S::KD + 8 * lane);
+      const uint2 dvr = *reinterpret_cast<const uint2 *>(st + S::VD + 8 * lane);
+      const float2 dk01 = __half22float2(*reinterpret_cast<const __half2 *>(&dkr.x));
+      const float2 dk23 = __half22float2(*reinterpret_cast<const __half2 *>(&dkr.y));
+      const float2 dv01 = __half22float2(*reinterpret_cast<const __half2 *>(&dvr.x));
+      const float2 dv23 = __half22float2(*reinterpret_cast<const __half2 *>(&dvr.y));
+      float tkl = 1.f, tvl = 1.f;
+      if (FAM == FAM_KVARN) {
+        tkl = h2f(reinterpret_cast<const __half *>(st + S::KT), lane);
+        tvl = h2f(reinterpret_cast<const __half *>(st + S::VT), lane);
+      }
+      // select (not multiply) so that NaN bit patterns in stale rows cannot leak
+      const float dkt[4] = {vl ? dk01.x * tkl : 0.f, vl ? dk01.y * tkl : 0.f, vl ? dk23.x * tkl : 0.f,
+                            vl ? dk23.y * tkl : 0.f};
+      *reinterpret_cast<float4 *>(&T.k[lane][0]) = make_float4(dkt[0], dkt[1], dkt[2], dkt[3]);
+      float tdv[4] = {vl ? dv01.x * tvl : 0.f, vl ? dv01.y * tvl : 0.f, vl ? dv23.x * tvl : 0.f,
+                      vl ? dv23.y * tvl : 0.f};
+      float inv[4];
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        float mx = tdv[blk];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+        inv[blk] = mx > 0.f ? QFIX * __frcp_rn(mx) : 0.f;
+        scl[blk] = mx * SCL;
+      }
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) T.v[blk][lane] = tdv[blk] * inv[blk];
+      if (FAM == FAM_ASYM) {
+        const uint2 mkr = *reinterpret_cast<const uint2 *>(st + S::KM + 8 * lane);
+        const uint2 mvr = *reinterpret_cast<const uint2 *>(st + S::VM + 8 * lane);
+        const float2 mk01 = __half22float2(*reinterpret_cast<const __half2 *>(&mkr.x));
+        const float2 mk23 = __half22float2(*reinterpret_cast<const __half2 *>(&mkr.y));
+        const float2 mv01 = __half22float2(*reinterpret_cast<const __half2 *>(&mvr.x));
+        const float2 mv23 = __half22float2(*reinterpret_cast<const __half2 *>(&mvr.y));
+        *reinterpret_cast<float4 *>(&T.km[lane][0]) =
+            make_float4(vl ? fmaf(dk01.x, HALF_RANGE, mk01.x) : 0.f, vl ? fmaf(dk01.y, HALF_RANGE, mk01.y) : 0.f,
+                        vl ? fmaf(dk23.x, HALF_RANGE, mk23.x) : 0.f, vl ? fmaf(dk23.y, HALF_RANGE, mk23.y) : 0.f);
+        *reinterpret_cast<float4 *>(&T.vm[lane][0]) =
+            make_float4(vl ? fmaf(dv01.x, HALF_RANGE, mv01.x) : 0.f, vl ? fmaf(dv01.y, HALF_RANGE, mv01.y) : 0.f,
+                        vl ? fmaf(dv23.x, HALF_RANGE, mv23.x) : 0.f, vl ? fmaf(dv23.y, HALF_RANGE, mv23.y) : 0.f);
+      }
+      __syncwarp();
+    }
 
     // ---- Q.K: n-tile r, column n holds token 16(r>>1) + 4(n>>1) + 2(r&1) + (n&1), so that
     //      the lane ends with the scores of tokens 4tq+(0..3) and 16+4tq+(0..3)
@@ -374,26 +429,28 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     for (int r = 0; r < 4; ++r) {
       KTok<FAM, BITS> kt;
       kt.load(st + S::KC + (16 * (r >> 1) + 4 * (g >> 1) + 2 * (r & 1) + (g & 1)) * 16 * BITS, tq);
-      float x0 = 0.f, x1 = 0.f, o0 = 0.f, o1 = 0.f;
       const int t0 = 16 * (r >> 1) + 4 * tq + 2 * (r & 1);
+      const float4 dA = *reinterpret_cast<const float4 *>(&T.k[t0][0]);
+      const float4 dB = *reinterpret_cast<const float4 *>(&T.k[t0 + 1][0]);
+      const float d0[4] = {dA.x, dA.y, dA.z, dA.w}, d1[4] = {dB.x, dB.y, dB.z, dB.w};
+      float x0 = 0.f, x1 = 0.f;
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
         uint32_t b0, b1;
         kt.frag(blk, tq, b0, b1);
-        int c[4] = {0, 0, 0, 0};
-        mma_s8(c, qa[blk], b0, b1);
-        const float d0 = h2f(dk, t0 * 4 + blk), d1 = h2f(dk, (t0 + 1) * 4 + blk);
-        x0 = fmaf(d0, (float)(c[0] * 256 + c[2]), x0);
-        x1 = fmaf(d1, (float)(c[1] * 256 + c[3]), x1);
-        if (FAM == FAM_ASYM) {
-          o0 = fmaf(fmaf(d0, HALF_RANGE, h2f(mk, t0 * 4 + blk)), qs[blk], o0);
-          o1 = fmaf(fmaf(d1, HALF_RANGE, h2f(mk, (t0 + 1) * 4 + blk)), qs[blk], o1);
-        }
+        int c[4];
+        mma_s8_bias(c, qa[blk], b0, b1, kBias);
+        const float h0 = __int_as_float(c[0]) - kBiasF, h1 = __int_as_float(c[1]) - kBiasF;
+        const float l0 = __int_as_float(c[2]) - kBiasF, l1 = __int_as_float(c[3]) - kBiasF;
+        x0 = fmaf(d0[blk], fmaf(256.f, h0, l0), x0);
+        x1 = fmaf(d1[blk], fmaf(256.f, h1, l1), x1);
       }
-      float s0 = x0 * sigp + o0, s1 = x1 * sigp + o1;
-      if (FAM == FAM_KVARN) {
-        s0 *= h2f(tk, t0);
-        s1 *= h2f(tk, t0 + 1);
+      float s0 = x0 * sigp, s1 = x1 * sigp;
+      if (FAM == FAM_ASYM) {
+        const float4 mA = *reinterpret_cast<const float4 *>(&T.km[t0][0]);
+        const float4 mB = *reinterpret_cast<const float4 *>(&T.km[t0 + 1][0]);
+        s0 = fmaf(mA.x, qs[0], fmaf(mA.y, qs[1], fmaf(mA.z, qs[2], fmaf(mA.w, qs[3], s0))));
+        s1 = fmaf(mB.x, qs[0], fmaf(mB.y, qs[1], fmaf(mB.z, qs[2], fmaf(mB.w, qs[3], s1))));
       }
       sc[2 * r] = t0 < nvalid ? s0 : -INFINITY;
       sc[2 * r + 1] = t0 + 1 < nvalid ? s1 : -INFINITY;
@@ -415,42 +472,32 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     }
     if (alpha != 1.f) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        acc[i] *= alpha;
-        accp[i] *= alpha;
-      }
+      for (int i = 0; i < 32; ++i) acc[i] *= alpha;
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) aoff[blk] *= alpha;
     }
     l_run = l_run * alpha + psum;
     m_run = mn;
 
-    // ---- P.V: weights w = p * t * d per (token, block) in 16-bit fixed point, scaled per
-    //      block by the chunk's largest t*d (p <= 1); rows past the end of the context may
-    //      hold stale bytes and are kept out of every sum
-#pragma unroll
-    for (int blk = 0; blk < 4; ++blk) {
-      float td[8], tdm = 0.f;
+    // ---- P.V: weights p * (t d QFIX / max) in 16-bit fixed point, two int8 limbs
+    if (FAM == FAM_ASYM) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const int tok = 16 * (k >> 2) + 4 * tq + (k & 3);
-        const bool vk = tok < nvalid;
-        float v = h2f(dvv, tok * 4 + blk);
-        if (FAM == FAM_KVARN) v *= h2f(tvv, tok);
-        v = vk ? v : 0.f;
-        td[k] = v;
-        tdm = fmaxf(tdm, v);
-        if (FAM == FAM_ASYM) {
-          const float mv = vk ? h2f(mvv, tok * 4 + blk) : 0.f;
-          aoff[blk] = fmaf(p[k], fmaf(v, HALF_RANGE, mv), aoff[blk]);
-        }
+        const float4 m4 = *reinterpret_cast<const float4 *>(&T.vm[16 * (k >> 2) + 4 * tq + (k & 3)][0]);
+        aoff[0] = fmaf(p[k], m4.x, aoff[0]);
+        aoff[1] = fmaf(p[k], m4.y, aoff[1]);
+        aoff[2] = fmaf(p[k], m4.z, aoff[2]);
+        aoff[3] = fmaf(p[k], m4.w, aoff[3]);
       }
-      tdm = fmaxf(tdm, __shfl_xor_sync(FULL, tdm, 1));
-      tdm = fmaxf(tdm, __shfl_xor_sync(FULL, tdm, 2));
-      const float inv = tdm > 0.f ? QFIX / tdm : 0.f;
+    }
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      const float4 ta = *reinterpret_cast<const float4 *>(&T.v[blk][4 * tq]);
+      const float4 tb = *reinterpret_cast<const float4 *>(&T.v[blk][16 + 4 * tq]);
+      const float tvk[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
       uint32_t wb[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) wb[k] = __float_as_uint(fmaf(p[k], td[k] * inv, MAGIC));
+      for (int k = 0; k < 8; ++k) wb[k] = __float_as_uint(fmaf(p[k], tvk[k], MAGIC));
       uint32_t wa[4];
       {
         const uint32_t x = __byte_perm(wb[0], wb[1], 0x5140), y = __byte_perm(wb[2], wb[3], 0x5140);
@@ -462,45 +509,40 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
         wa[2] = __byte_perm(x, y, 0x7632);
         wa[3] = __byte_perm(x, y, 0x5410) ^ 0x80808080u;
       }
+      // per-channel factor: the block's fixed-point scale, times the page's V channel scale c
+      float f[8];
+      if (FAM == FAM_KVARN) {
+        const uint4 c8 = *reinterpret_cast<const uint4 *>(st + S::VCS + 2 * (32 * blk + 8 * tq));
+        const __half2 *c2 = reinterpret_cast<const __half2 *>(&c8);
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) {
+          const float2 cf = __half22float2(c2[q2]);
+          f[2 * q2] = scl[blk] * cf.x;
+          f[2 * q2 + 1] = scl[blk] * cf.y;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = scl[blk];
+      }
       VQuad<FAM, BITS> v0, v1;
       v0.load(st + S::VC + tq * S::QS, blk, g);
       v1.load(st + S::VC + (4 + tq) * S::QS, blk, g);
-      const float scl = tdm / QFIX * CSC;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        int c[4] = {0, 0, 0, 0};
-        mma_s8(c, wa, v0.frag(u, g), v1.frag(u, g));
-        float *dst = FAM == FAM_KVARN ? accp : acc;
-        dst[blk * 8 + u * 2 + 0] = fmaf(scl, (float)(c[0] * 256 + c[2]), dst[blk * 8 + u * 2 + 0]);
-        dst[blk * 8 + u * 2 + 1] = fmaf(scl, (float)(c[1] * 256 + c[3]), dst[blk * 8 + u * 2 + 1]);
+        int c[4];
+        mma_s8_bias(c, wa, v0.frag(u, g), v1.frag(u, g), kBias);
+        const float h0 = __int_as_float(c[0]) - kBiasF, h1 = __int_as_float(c[1]) - kBiasF;
+        const float l0 = __int_as_float(c[2]) - kBiasF, l1 = __int_as_float(c[3]) - kBiasF;
+        // column 2tq <-> channel 32 blk + 8 tq + u, column 2tq+1 <-> + 4
+        acc[blk * 8 + u * 2 + 0] = fmaf(f[u], fmaf(256.f, h0, l0), acc[blk * 8 + u * 2 + 0]);
+        acc[blk * 8 + u * 2 + 1] = fmaf(f[4 + u], fmaf(256.f, h1, l1), acc[blk * 8 + u * 2 + 1]);
       }
     }
 
-    // kvarn: at the last chunk of a page fold the page's V channel scales c into acc
-    if (FAM == FAM_KVARN && (j + 1 == nj || (a + (c0 + j + 1) * CH) / GROUP != page)) {
-      const __half *cv = reinterpret_cast<const __half *>(st + S::VCS);
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk)
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int idx = blk * 8 + u * 2 + e;
-            acc[idx] = fmaf(h2f(cv, 32 * blk + 8 * tq + 4 * e + u), accp[idx], acc[idx]);
-            accp[idx] = 0.f;
-          }
-    }
-
-    __syncwarp();
-    if (lane == 0 && j + S::NST < nj) {
-      fence_proxy_async();  // this warp's reads of the stage come before the copy into it
-      issue_chunk<FAM, BITS>(L, seq, head, a + (c0 + j + S::NST) * CH, st, &bars[si]);
-    }
+    __syncwarp();  // every lane is done with stage si before it is refilled next round
   }
-  if (!ok) {
-    // drain: wait (bounded) for every copy still in flight before the stage memory is reused
-    for (int j = 0; j < nj && j < S::NST; ++j) mbar_wait(&bars[j], 0u, L.status);
-  }
+  cp_async_wait<0>();
+  __syncwarp();
   l_run += __shfl_xor_sync(FULL, l_run, 1);
   l_run += __shfl_xor_sync(FULL, l_run, 2);
   if (FAM == FAM_ASYM) {
@@ -542,6 +584,7 @@ __device__ __forceinline__ void warp_bf16(const LayerView &L, int seq, int head,
   }
   const __nv_bfloat16 *kbase = ring_row(L, seq, head, 0, 0);
   const __nv_bfloat16 *vbase = ring_row(L, seq, head, 1, 0);
+#pragma unroll 1
   for (int64_t ci = c0; ci < c1; ++ci) {
     const int64_t i0 = a + ci * CH;
     const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
@@ -635,8 +678,38 @@ __device__ __forceinline__ void warp_bf16(const LayerView &L, int seq, int head,
   }
 }
 
+// H.x of one 128-wide row by one warp: the lane holds x[4 lane .. 4 lane + 3]; butterfly
+// stages h = 1, 2 inside the lane, h = 4 .. 64 across lanes (xor 1 .. 16)
+__device__ __forceinline__ void warp_wht(float (&v)[4], int lane) {
+  float a = v[0], b = v[1];
+  v[0] = a + b;
+  v[1] = a - b;
+  a = v[2];
+  b = v[3];
+  v[2] = a + b;
+  v[3] = a - b;
+  a = v[0];
+  b = v[2];
+  v[0] = a + b;
+  v[2] = a - b;
+  a = v[1];
+  b = v[3];
+  v[1] = a + b;
+  v[3] = a - b;
+#pragma unroll
+  for (int o = 1; o <= 16; o <<= 1) {
+    const bool hi = lane & o;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float other = __shfl_xor_sync(FULL, v[e], o);
+      v[e] = hi ? other - v[e] : v[e] + other;
+    }
+  }
+}
+
 // Shared memory of the kernel (dynamic): fixed part + per-warp stage area (also used for the
 // warps' accumulators once the chunks are done).
+template <int NW>
 struct SmemFixed {
   float qraw[MAX_G][D];
   float qrot[MAX_G][D];
@@ -646,7 +719,8 @@ struct SmemFixed {
   float fl[MAXSPL][MAX_G];   // merge: l of each split
   float red[MAX_G][D];       // merge: second half of the split sum
   float Ls[MAX_G];
-  uint64_t bars[NW][4];
+  float Mc[MAX_G], Lc[MAX_G];  // this CTA's combined m and l per head
+  ChunkTabs tabs[NW];
   int is_last;
 };
 
@@ -662,14 +736,16 @@ __host__ __device__ constexpr int warp_area() {
 
 template <int FAM, int BITS>
 __host__ __device__ constexpr size_t smem_bytes() {
-  return ((sizeof(SmemFixed) + 127) / 128) * 128 + (size_t)NW * warp_area<FAM, BITS>();
+  constexpr int NW = nwarps(FAM, BITS);
+  return ((sizeof(SmemFixed<NW>) + 127) / 128) * 128 + (size_t)NW * warp_area<FAM, BITS>();
 }
 
 template <int FAM, int BITS>
-__global__ void __launch_bounds__(DT, 1) k_decode(LayerView L, DArgs A) {
+__global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView L, DArgs A) {
+  constexpr int NW = nwarps(FAM, BITS), DT = 32 * NW;
   extern __shared__ __align__(128) uint8_t smem[];
-  SmemFixed &F = *reinterpret_cast<SmemFixed *>(smem);
-  uint8_t *warp_mem = smem + ((sizeof(SmemFixed) + 127) / 128) * 128;
+  SmemFixed<NW> &F = *reinterpret_cast<SmemFixed<NW> *>(smem);
+  uint8_t *warp_mem = smem + ((sizeof(SmemFixed<NW>) + 127) / 128) * 128;
   constexpr int WA = warp_area<FAM, BITS>();
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -696,10 +772,6 @@ __global__ void __launch_bounds__(DT, 1) k_decode(LayerView L, DArgs A) {
   const int64_t per = (nch + NW - 1) / NW;
   const int64_t c0 = min((int64_t)warp * per, nch), c1 = min(c0 + per, nch);
 
-  if (lane == 0 && FAM != FAM_BF16 && !tail) {
-    for (int j = 0; j < 4; ++j) mbar_init(&F.bars[warp][j], 1);
-    fence_proxy_async();
-  }
   // query rows of this KV head, pre-scaled by softmax_scale * log2(e); heads >= G are 0
   for (int idx = tid; idx < MAX_G * D; idx += DT) {
     const int g = idx / D, j = idx % D;
@@ -711,23 +783,14 @@ __global__ void __launch_bounds__(DT, 1) k_decode(LayerView L, DArgs A) {
   }
   __syncthreads();
   if (!tail && A.rotk) {
-    // q' = H.q.kappa with the same butterfly as the keys' rotation
-    if (tid < G) {
-      float r[D];
+    // q' = H.q.kappa, one warp per query head
+    if (warp < G) {
+      float v[4];
 #pragma unroll
-      for (int j = 0; j < D; ++j) r[j] = F.qraw[tid][j];
+      for (int e = 0; e < 4; ++e) v[e] = F.qraw[warp][4 * lane + e];
+      warp_wht(v, lane);
 #pragma unroll
-      for (int h = 1; h < D; h <<= 1) {
-#pragma unroll
-        for (int j = 0; j < D; ++j) {
-          if (j & h) continue;
-          const float x = r[j], y = r[j + h];
-          r[j] = x + y;
-          r[j + h] = x - y;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < D; ++j) F.qrot[tid][j] = r[j] * kKappa();
+      for (int e = 0; e < 4; ++e) F.qrot[warp][4 * lane + e] = v[e] * kKappa();
     }
   } else {
     for (int idx = tid; idx < MAX_G * D; idx += DT) F.qrot[idx / D][idx % D] = F.qraw[idx / D][idx % D];
@@ -737,7 +800,7 @@ __global__ void __launch_bounds__(DT, 1) k_decode(LayerView L, DArgs A) {
   float *accw = reinterpret_cast<float *>(warp_mem + (size_t)warp * WA);  // [MAX_G][D] after the chunks
   if constexpr (FAM != FAM_BF16) {
     if (!tail) {
-      warp_quant<FAM, BITS>(L, s.seq, head, a, b, c0, c1, G, F.qrot, warp_mem + (size_t)warp * WA, F.bars[warp],
+      warp_quant<FAM, BITS>(L, s.seq, head, a, b, c0, c1, G, F.qrot, warp_mem + (size_t)warp * WA, F.tabs[warp],
                             F.mw[warp], F.lw[warp], accw);
     } else {
       for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
@@ -753,25 +816,30 @@ __global__ void __launch_bounds__(DT, 1) k_decode(LayerView L, DArgs A) {
 
   // combine the warps of this CTA into its partial (m, l, acc) per query head
   const int slot0 = s.part0 + head * nspl;
-  if (tid < D) {
-    for (int g = 0; g < G; ++g) {
-      float M = -INFINITY;
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, F.mw[w][g]);
-      float av = 0.f, lv = 0.f;
-      if (M != -INFINITY) {
-        for (int w = 0; w < NW; ++w) {
-          if (F.mw[w][g] == -INFINITY) continue;
-          const float f = exp2f(F.mw[w][g] - M);
-          av += f * reinterpret_cast<const float *>(warp_mem + (size_t)w * WA)[g * D + tid];
-          lv += f * F.lw[w][g];
-        }
-      }
-      float *dst = A.ws + ((int64_t)(slot0 + sp) * G + g) * PSTRIDE;
-      dst[2 + tid] = av;
-      if (tid == 0) {
-        dst[0] = M;
-        dst[1] = lv;
-      }
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, F.mw[w][tid]);
+    float lsum = 0.f;
+    for (int w = 0; w < NW; ++w) {
+      const float f = (M == -INFINITY || F.mw[w][tid] == -INFINITY) ? 0.f : exp2f(F.mw[w][tid] - M);
+      F.fw[w][tid] = f;
+      lsum = fmaf(f, F.lw[w][tid], lsum);
+    }
+    F.Mc[tid] = M;
+    F.Lc[tid] = lsum;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < G * D; idx += DT) {
+    const int g = idx / D, c = idx % D;
+    float av = 0.f;
+#pragma unroll 4
+    for (int w = 0; w < NW; ++w)
+      av = fmaf(F.fw[w][g], reinterpret_cast<const float *>(warp_mem + (size_t)w * WA)[g * D + c], av);
+    float *dst = A.ws + ((int64_t)(slot0 + sp) * G + g) * PSTRIDE;
+    dst[2 + c] = av;
+    if (c == 0) {
+      dst[0] = F.Mc[g];
+      dst[1] = F.Lc[g];
     }
   }
 
@@ -804,45 +872,67 @@ __global__ void __launch_bounds__(DT, 1) k_decode(LayerView L, DArgs A) {
     F.Ls[tid] = Ls;
   }
   __syncthreads();
-  // thread = (half, channel): half 0 sums the quantized splits (stored basis), half 1 the
-  // tail splits (original basis)
-  const int ch = tid & (D - 1), half = tid >> 7;
-  const int k0 = half == 0 ? 0 : s.nsq, k1 = half == 0 ? s.nsq : nspl;
-  float sum[MAX_G];
+  // thread = (group, channel): group r sums splits r, r + NGR, ... for every head, the loads
+  // of a batch of splits all issued before any is used; quantized splits (stored basis) and
+  // tail splits (original basis) are kept apart
+  constexpr int NGR = DT / D;  // 2 or 3 groups of 128 threads
+  constexpr int KB = 4;        // splits per batch and thread
+  const int ch = tid & (D - 1), grp = tid / D;
+  float srot[MAX_G], spl[MAX_G];
 #pragma unroll
-  for (int g = 0; g < MAX_G; ++g) sum[g] = 0.f;
-  for (int k = k0; k < k1; ++k) {
+  for (int g = 0; g < MAX_G; ++g) srot[g] = spl[g] = 0.f;
+  for (int kb = grp; kb < nspl; kb += NGR * KB) {
+    float v[KB][MAX_G];
 #pragma unroll
-    for (int g = 0; g < MAX_G; ++g)
-      if (g < G) sum[g] = fmaf(F.fw[k][g], __ldcg(part + ((int64_t)k * G + g) * PSTRIDE + 2 + ch), sum[g]);
-  }
-  if (half == 0) {
+    for (int u = 0; u < KB; ++u) {
+      const int k = kb + u * NGR;
 #pragma unroll
-    for (int g = 0; g < MAX_G; ++g)
-      if (g < G) F.qraw[g][ch] = sum[g];  // q rows are no longer needed
-  } else {
+      for (int g = 0; g < MAX_G; ++g)
+        v[u][g] = (k < nspl && g < G) ? __ldcg(part + ((int64_t)k * G + g) * PSTRIDE + 2 + ch) : 0.f;
+    }
 #pragma unroll
-    for (int g = 0; g < MAX_G; ++g)
-      if (g < G) F.red[g][ch] = sum[g];
-  }
-  __syncthreads();
-  if (A.rotv) {
-    // inverse rotation of the quantized part of every head: H.acc.kappa
-    for (int h = 1; h < D; h <<= 1) {
-      for (int idx = tid; idx < G * D / 2; idx += DT) {
-        const int g = idx / (D / 2), pr = idx % (D / 2);
-        const int lo = (pr / h) * 2 * h + (pr % h);
-        const float x = F.qraw[g][lo], y = F.qraw[g][lo + h];
-        F.qraw[g][lo] = x + y;
-        F.qraw[g][lo + h] = x - y;
+    for (int u = 0; u < KB; ++u) {
+      const int k = kb + u * NGR;
+      if (k >= nspl) break;
+#pragma unroll
+      for (int g = 0; g < MAX_G; ++g) {
+        if (g >= G) break;
+        if (k < s.nsq)
+          srot[g] = fmaf(F.fw[k][g], v[u][g], srot[g]);
+        else
+          spl[g] = fmaf(F.fw[k][g], v[u][g], spl[g]);
       }
-      __syncthreads();
     }
   }
-  for (int idx = tid; idx < G * D; idx += DT) {
-    const int g = idx / D, c = idx % D;
-    const float rot = A.rotv ? F.qraw[g][c] * kKappa() : F.qraw[g][c];
-    A.out[((int64_t)s.row * A.hkv * G + head * G + g) * D + c] = F.Ls[g] > 0.f ? (rot + F.red[g][c]) / F.Ls[g] : 0.f;
+  // combine the groups: F.red[g] holds the plain sums, F.qraw[g] the stored-basis sums
+  for (int r = 0; r < NGR; ++r) {
+    if (grp == r) {
+#pragma unroll
+      for (int g = 0; g < MAX_G; ++g) {
+        if (g >= G) break;
+        F.qraw[g][ch] = (r == 0 ? 0.f : F.qraw[g][ch]) + srot[g];
+        F.red[g][ch] = (r == 0 ? 0.f : F.red[g][ch]) + spl[g];
+      }
+    }
+    __syncthreads();
+  }
+  // output: (H.acc_rot.kappa + acc_plain) / L, one warp per query head
+  for (int g = warp; g < G; g += NW) {
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = F.qraw[g][4 * lane + e];
+    if (A.rotv) {
+      warp_wht(v, lane);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] *= kKappa();
+    }
+    const float Lg = F.Ls[g];
+    float4 o;
+    o.x = Lg > 0.f ? (v[0] + F.red[g][4 * lane + 0]) / Lg : 0.f;
+    o.y = Lg > 0.f ? (v[1] + F.red[g][4 * lane + 1]) / Lg : 0.f;
+    o.z = Lg > 0.f ? (v[2] + F.red[g][4 * lane + 2]) / Lg : 0.f;
+    o.w = Lg > 0.f ? (v[3] + F.red[g][4 * lane + 3]) / Lg : 0.f;
+    *reinterpret_cast<float4 *>(A.out + ((int64_t)s.row * A.hkv * G + head * G + g) * D + 4 * lane) = o;
   }
   if (tid == 0) A.tickets[s.seq * A.hkv + head] = 0u;
 }
@@ -857,7 +947,7 @@ cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_decode<FAM, BITS><<<A.ncta, DT, smem, st>>>(L, A);
+  k_decode<FAM, BITS><<<A.ncta, 32 * nwarps(FAM, BITS), smem, st>>>(L, A);
   return cudaGetLastError();
 }
 
