@@ -227,6 +227,7 @@ struct KvarnSmem {
   float part[8][GROUP]; // token-sum partials of the 8 channel runs
   float rc[D];          // 1/fp16(c)
   float rt[GROUP];      // 1/fp16(t)
+  uint32_t img[GROUP * 16 * 8 / 4];  // packed code area of the sub-page (up to 8-bit codes)
 };
 
 // d = a*b + c on two fp32 lanes, each rounded once (the same result as two fmaf)
@@ -239,6 +240,104 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   float2 d;
   memcpy(&d, &rd, 8);
   return d;
+}
+
+// Thread-per-token quantization of a balanced group (see k_spill_kvarn, step 4).  The block
+// loop is kept rolled: the kernel is long straight-line code executed once per CTA, so its
+// instruction footprint, not its arithmetic, sets the pace.
+template <int BITS, int WHICH>
+__device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const SubLayout &lay, int ng, int tid) {
+  constexpr int QMAX = (1 << (BITS - 1)) - 1, QMIN = -(1 << (BITS - 1));
+  constexpr int WL = plane_lo(BITS), WH = plane_hi(BITS);
+  uint8_t *img = reinterpret_cast<uint8_t *>(S.img);
+  if (tid < ng) {
+    const float rti = S.rt[tid];
+    uint32_t dlo = 0u, dhi = 0u;
+#pragma unroll 1
+    for (int blk = 0; blk < 4; ++blk) {
+      float y[32];
+      float amax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        y[e] = __fmul_rn(__fmul_rn(S.X[tid * XS + 32 * blk + e], S.rc[32 * blk + e]), rti);
+        amax = fmaxf(amax, fabsf(y[e]));
+      }
+      const __half dh = sat_half(__fdiv_rn(amax, (float)QMAX));
+      const float df = __half2float(dh);
+      const float rd = df != 0.0f ? __frcp_rn(df) : 0.0f;
+      const uint32_t dv = (uint32_t)__half_as_ushort(dh) << (16 * (blk & 1));
+      if (blk < 2)
+        dlo |= dv;
+      else
+        dhi |= dv;
+      // rint(RN(y/d)) by the reciprocal; the exact quotient only where a value sits within 4 ulp
+      // of a half-integer (checked once for the block)
+      float r[32];
+      bool tie = false;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float q = __fmul_rn(y[e], rd);
+        r[e] = rintf(q);
+        const float tol = fmaxf(fabsf(q), 1.0f) * 9.5367431640625e-07f;
+        tie |= fabsf(fabsf(__fsub_rn(q, r[e])) - 0.5f) <= tol;
+      }
+      if (tie) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = rintf(__fdiv_rn(y[e], df));
+      }
+      uint32_t f[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float rr = df != 0.0f ? fminf(fmaxf(r[e], (float)QMIN), (float)QMAX) : 0.0f;
+        f[e] = (uint32_t)(int)rr & ((1u << BITS) - 1u);
+      }
+#pragma unroll
+      for (int pl = 0; pl < 2; ++pl) {
+        const int w = pl == 0 ? WL : WH;
+        if (w == 0) continue;
+        const int shift_in = pl == 0 ? 0 : WL;
+        const uint32_t wm = (1u << w) - 1u;
+        const int F = 8 / w;
+        if (WHICH == 0) {
+          // K: channel 32 blk + 4 jj + k -> byte k of word (jj / F, blk), bits (jj % F) w
+          uint8_t *plane = img + tid * 16 * BITS + (pl == 0 ? 0 : 16 * WL);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            if (m >= w) break;
+            uint32_t word = 0;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              if (jj / F != m) continue;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                word |= ((f[4 * jj + kk] >> shift_in) & wm) << (8 * kk + (jj % F) * w);
+            }
+            *reinterpret_cast<uint32_t *>(plane + 16 * m + 4 * blk) = word;
+          }
+        } else {
+          // V: channel 32 blk + e of quad token k -> byte k of word e / F of block blk,
+          // bits (e % F) w
+          uint8_t *plane = img + (tid >> 2) * 64 * BITS + (pl == 0 ? 0 : 64 * WL) + 16 * w * blk + (tid & 3);
+#pragma unroll
+          for (int m = 0; m < 32; ++m) {
+            if (m >= 4 * w) break;
+            uint32_t byte = 0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (e / F != m) continue;
+              byte |= ((f[e] >> shift_in) & wm) << ((e % F) * w);
+            }
+            plane[4 * m] = (uint8_t)byte;
+          }
+        }
+      }
+    }
+    *reinterpret_cast<uint2 *>(sub + lay.d + tid * 8) = make_uint2(dlo, dhi);
+  }
+  __syncthreads();
+  const int nbytes = WHICH == 0 ? ng * 16 * BITS : ((ng + 3) / 4) * 64 * BITS;
+  for (int p = tid; p < nbytes / 16; p += KV_THREADS)
+    reinterpret_cast<uint4 *>(sub)[p] = reinterpret_cast<const uint4 *>(img)[p];
 }
 
 // One CTA (256 threads) per (kvarn group, head, K or V).  Per sequence, s.a is the first
@@ -427,19 +526,13 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
   }
   __syncthreads();
 
-  // 4. y = (x * rc_j) * rt_i, symmetric b-bit blocks of 32, packed
-  const float4 rc4 = *reinterpret_cast<const float4 *>(&S.rc[4 * lane]);
-  const float rcl[4] = {rc4.x, rc4.y, rc4.z, rc4.w};
-  for (int i = warp; i < ng; i += 8) {
-    float y[4];
-    const float rti = S.rt[i];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) y[e] = __fmul_rn(__fmul_rn(S.X[i * XS + 4 * lane + e], rcl[e]), rti);
-    if (which == 0)
-      quant_sym<BITS, 0>(y, sub, lay, i, lane);
-    else
-      quant_sym<BITS, 1>(y, sub, lay, i, lane);
-  }
+  // 4. thread i quantizes token i: y = (x * rc_j) * rt_i, symmetric b-bit blocks of 32; the
+  //    packed codes go to an image of the sub-page's code area in shared memory (it reuses
+  //    the tile), which the CTA then copies out with 16-byte stores
+  if (which == 0)
+    quant_rows<BITS, 0>(S, sub, lay, ng, tid);
+  else
+    quant_rows<BITS, 1>(S, sub, lay, ng, tid);
 }
 
 // Copies new rows that stay 16-bit into the ring: range per sequence [a, n1), rows

@@ -194,6 +194,13 @@ __device__ __forceinline__ uint32_t pack_s8(int a, int b, int c, int d) {
 
 __device__ __forceinline__ float h2f(const __half *p, int i) { return __half2float(p[i]); }
 
+// 2^x by the MUFU unit (flushes results below 2^-126 to 0: negligible softmax weights)
+__device__ __forceinline__ float exp2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 constexpr float QFIX = 32639.0f;              // 16-bit fixed point: 256*127 + 127
 constexpr float MAGIC = 12582912.0f + 128.0f;  // 1.5*2^23 (+128 offset for the limb split)
 
@@ -463,11 +470,11 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 1));
     cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 2));
     const float mn = fmaxf(m_run, cmax);
-    const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mn);
+    const float alpha = m_run == -INFINITY ? 0.f : exp2_fast(m_run - mn);
     float p[8], psum = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      p[k] = sc[k] == -INFINITY ? 0.f : exp2f(sc[k] - mn);
+      p[k] = sc[k] == -INFINITY ? 0.f : exp2_fast(sc[k] - mn);
       psum += p[k];
     }
     if (alpha != 1.f) {
@@ -632,8 +639,8 @@ __device__ __forceinline__ void warp_bf16(const LayerView &L, int seq, int head,
       if (g >= G) break;
       const float sv_ = valid ? sc[g] : -INFINITY;
       const float mn = fmaxf(m[g], warp_max(sv_));
-      const float alpha = m[g] == -INFINITY ? 0.f : exp2f(m[g] - mn);
-      const float p = valid ? exp2f(sv_ - mn) : 0.f;
+      const float alpha = m[g] == -INFINITY ? 0.f : exp2_fast(m[g] - mn);
+      const float p = valid ? exp2_fast(sv_ - mn) : 0.f;
       l[g] = l[g] * alpha + warp_sum(p);
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[g][e] *= alpha;
