@@ -30,7 +30,8 @@ constexpr int CH = 32;       // tokens per chunk (one per lane)
 constexpr int MAXSQ = 48;    // max splits over the quantized prefix per (seq, head)
 constexpr int MAXST = 16;    // max splits over the tail per (seq, head)
 constexpr int MAXSPL = MAXSQ + MAXST;
-constexpr int PSTRIDE = 2 + D;  // floats per partial: m, l, acc[128]
+constexpr int PSTRIDE = 4 + D;  // floats per partial: m, l, 2 pad, acc[128] (16-byte records)
+constexpr int PACC = 4;         // offset of acc in a partial
 constexpr int MAXS = 64;        // sequences per launch
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -291,6 +292,19 @@ struct ChunkTabs {
 constexpr int kBias = 0x4B400000;       // float bits of 1.5 * 2^23
 constexpr float kBiasF = 12582912.0f;  // an int32 accumulator started at kBias reads as kBiasF + sum
 
+// Issues the first NST - 1 chunks of a warp's range (one commit group each, empty groups past
+// the end), so that their copies overlap the query prologue.
+template <int FAM, int BITS>
+__device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq, int head, int64_t a, int64_t c0,
+                                                    int64_t c1, uint8_t *stages, int lane) {
+  using S = Stage<FAM, BITS>;
+#pragma unroll
+  for (int j = 0; j < S::NST - 1; ++j) {
+    if (j < c1 - c0) copy_chunk<FAM, BITS>(L, seq, head, a + (c0 + j) * CH, stages + j * S::BYTES, lane);
+    cp_async_commit();
+  }
+}
+
 // Q.K and P.V of one warp over its chunks [c0, c1) of a quantized split starting at token a
 // (chunks are consecutive, so pages change rarely).  Writes the warp's online-softmax state
 // (m, l and the accumulator in the stored basis) of its heads to shared memory.
@@ -316,12 +330,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
   int64_t cur_page = -1;
 
   const int nj = (int)(c1 - c0);
-  // prologue: NST - 1 chunks in flight (one commit group each, empty groups past the end)
-#pragma unroll
-  for (int j = 0; j < S::NST - 1; ++j) {
-    if (j < nj) copy_chunk<FAM, BITS>(L, seq, head, a + (c0 + j) * CH, stages + j * S::BYTES, lane);
-    cp_async_commit();
-  }
+  // the first NST - 1 chunks are already in flight (warp_quant_prefetch)
 #pragma unroll 1
   for (int j = 0; j < nj; ++j) {
     const int si = j % S::NST;
@@ -722,9 +731,10 @@ struct SmemFixed {
   float qrot[MAX_G][D];
   float pst[NW][CH][MAX_G];
   float mw[NW][MAX_G], lw[NW][MAX_G];
-  float fw[MAXSPL][MAX_G];   // merge: weight of each split
-  float fl[MAXSPL][MAX_G];   // merge: l of each split
-  float red[MAX_G][D];       // merge: second half of the split sum
+  float fw[MAXSPL][MAX_G];   // weight of each warp (CTA combine) / split (merge)
+  float fm[MAXSPL][MAX_G];   // merge: m and l of the splits whose records are not staged
+  float fl[MAXSPL][MAX_G];
+  float red[MAX_G][D];       // merge: sum over the tail splits (original basis)
   float Ls[MAX_G];
   float Mc[MAX_G], Lc[MAX_G];  // this CTA's combined m and l per head
   ChunkTabs tabs[NW];
@@ -734,7 +744,7 @@ struct SmemFixed {
 template <int FAM, int BITS>
 __host__ __device__ constexpr int warp_area() {
   if constexpr (FAM == FAM_BF16) {
-    return MAX_G * D * 4;
+    return 16384;  // accumulators, then (all warps together) the merge's staged partials
   } else {
     constexpr int s = Stage<FAM, BITS>::NST * Stage<FAM, BITS>::BYTES;
     return s > MAX_G * D * 4 ? s : MAX_G * D * 4;
@@ -779,6 +789,9 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
   const int64_t per = (nch + NW - 1) / NW;
   const int64_t c0 = min((int64_t)warp * per, nch), c1 = min(c0 + per, nch);
 
+  if constexpr (FAM != FAM_BF16) {
+    if (!tail) warp_quant_prefetch<FAM, BITS>(L, s.seq, head, a, c0, c1, warp_mem + (size_t)warp * WA, lane);
+  }
   // query rows of this KV head, pre-scaled by softmax_scale * log2(e); heads >= G are 0
   for (int idx = tid; idx < MAX_G * D; idx += DT) {
     const int g = idx / D, j = idx % D;
@@ -821,19 +834,19 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
   }
   __syncthreads();
 
-  // combine the warps of this CTA into its partial (m, l, acc) per query head
+  // combine the warps of this CTA into its partial (m, l, acc) per query head: warp g
+  // reduces head g over the warps, one lane per warp
   const int slot0 = s.part0 + head * nspl;
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, F.mw[w][tid]);
-    float lsum = 0.f;
-    for (int w = 0; w < NW; ++w) {
-      const float f = (M == -INFINITY || F.mw[w][tid] == -INFINITY) ? 0.f : exp2f(F.mw[w][tid] - M);
-      F.fw[w][tid] = f;
-      lsum = fmaf(f, F.lw[w][tid], lsum);
+  if (warp < G) {
+    const float mw = lane < NW ? F.mw[lane][warp] : -INFINITY;
+    const float M = warp_max(mw);
+    const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+    if (lane < NW) F.fw[lane][warp] = f;
+    const float lsum = warp_sum(lane < NW ? f * F.lw[lane][warp] : 0.f);
+    if (lane == 0) {
+      F.Mc[warp] = M;
+      F.Lc[warp] = lsum;
     }
-    F.Mc[tid] = M;
-    F.Lc[tid] = lsum;
   }
   __syncthreads();
   for (int idx = tid; idx < G * D; idx += DT) {
@@ -843,7 +856,7 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
     for (int w = 0; w < NW; ++w)
       av = fmaf(F.fw[w][g], reinterpret_cast<const float *>(warp_mem + (size_t)w * WA)[g * D + c], av);
     float *dst = A.ws + ((int64_t)(slot0 + sp) * G + g) * PSTRIDE;
-    dst[2 + c] = av;
+    dst[PACC + c] = av;
     if (c == 0) {
       dst[0] = F.Mc[g];
       dst[1] = F.Lc[g];
@@ -860,69 +873,75 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
   __syncthreads();
   if (!F.is_last) return;
   __threadfence();
+
+  // The partial records (nspl * G of them, contiguous) are staged in shared memory by cp.async,
+  // as many whole splits per batch as the warp areas hold; the m and l of the splits beyond
+  // the first batch are read directly, so that the weights are known before any sum.
   const float *part = A.ws + (int64_t)slot0 * G * PSTRIDE;
-  for (int idx = tid; idx < nspl * G; idx += DT) {
-    const float *src = part + (int64_t)idx * PSTRIDE;  // split idx / G, head idx % G
-    F.fw[idx / G][idx % G] = __ldcg(src);
-    F.fl[idx / G][idx % G] = __ldcg(src + 1);
+  float *stage = reinterpret_cast<float *>(warp_mem);
+  constexpr int CAP = (NW * WA) / (PSTRIDE * 4);  // records that fit
+  const int kper = CAP / G;                       // whole splits per batch (>= 1)
+  int kb0 = 0, kb1 = min(nspl, kper);
+  for (int p = tid; p < kb1 * G * (PSTRIDE / 4); p += DT) cp_async16(stage + 4 * p, part + 4 * p);
+  cp_async_commit();
+  for (int idx = kb1 * G + tid; idx < nspl * G; idx += DT) {
+    F.fm[idx / G][idx % G] = __ldcg(part + (int64_t)idx * PSTRIDE);
+    F.fl[idx / G][idx % G] = __ldcg(part + (int64_t)idx * PSTRIDE + 1);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  // split weights: warp g, one lane per split
+  if (warp < G) {
+    const int g = warp;
+    float mk[MAXSPL / 32], M = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < MAXSPL / 32; ++u) {
+      const int k = lane + 32 * u;
+      mk[u] = k < nspl ? (k < kb1 ? stage[(k * G + g) * PSTRIDE] : F.fm[k][g]) : -INFINITY;
+      M = fmaxf(M, mk[u]);
+    }
+    M = warp_max(M);
+    float ls = 0.f;
+#pragma unroll
+    for (int u = 0; u < MAXSPL / 32; ++u) {
+      const int k = lane + 32 * u;
+      if (k < nspl) {
+        const float f = (mk[u] == -INFINITY) ? 0.f : exp2f(mk[u] - M);
+        F.fw[k][g] = f;
+        ls = fmaf(f, k < kb1 ? stage[(k * G + g) * PSTRIDE + 1] : F.fl[k][g], ls);
+      }
+    }
+    ls = warp_sum(ls);
+    if (lane == 0) F.Ls[g] = ls;
   }
   __syncthreads();
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int k = 0; k < nspl; ++k) M = fmaxf(M, F.fw[k][tid]);
-    float Ls = 0.f;
-    for (int k = 0; k < nspl; ++k) {
-      const float f = (M == -INFINITY || F.fw[k][tid] == -INFINITY) ? 0.f : exp2f(F.fw[k][tid] - M);
-      F.fw[k][tid] = f;
-      Ls += f * F.fl[k][tid];
-    }
-    F.Ls[tid] = Ls;
-  }
-  __syncthreads();
-  // thread = (group, channel): group r sums splits r, r + NGR, ... for every head, the loads
-  // of a batch of splits all issued before any is used; quantized splits (stored basis) and
-  // tail splits (original basis) are kept apart
-  constexpr int NGR = DT / D;  // 2 or 3 groups of 128 threads
-  constexpr int KB = 4;        // splits per batch and thread
-  const int ch = tid & (D - 1), grp = tid / D;
-  float srot[MAX_G], spl[MAX_G];
-#pragma unroll
-  for (int g = 0; g < MAX_G; ++g) srot[g] = spl[g] = 0.f;
-  for (int kb = grp; kb < nspl; kb += NGR * KB) {
-    float v[KB][MAX_G];
-#pragma unroll
-    for (int u = 0; u < KB; ++u) {
-      const int k = kb + u * NGR;
-#pragma unroll
-      for (int g = 0; g < MAX_G; ++g)
-        v[u][g] = (k < nspl && g < G) ? __ldcg(part + ((int64_t)k * G + g) * PSTRIDE + 2 + ch) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < KB; ++u) {
-      const int k = kb + u * NGR;
-      if (k >= nspl) break;
-#pragma unroll
-      for (int g = 0; g < MAX_G; ++g) {
-        if (g >= G) break;
+  // weighted sums, one thread per (head, channel) output; quantized splits (stored basis)
+  // and tail splits (original basis) are kept apart
+  for (;;) {
+    for (int o = tid; o < G * D; o += DT) {
+      const int g = o / D, ch = o % D;
+      float srot = kb0 ? F.qraw[g][ch] : 0.f, spl = kb0 ? F.red[g][ch] : 0.f;
+      for (int k = kb0; k < kb1; ++k) {
+        const float v = stage[((k - kb0) * G + g) * PSTRIDE + PACC + ch];
         if (k < s.nsq)
-          srot[g] = fmaf(F.fw[k][g], v[u][g], srot[g]);
+          srot = fmaf(F.fw[k][g], v, srot);
         else
-          spl[g] = fmaf(F.fw[k][g], v[u][g], spl[g]);
+          spl = fmaf(F.fw[k][g], v, spl);
       }
+      F.qraw[g][ch] = srot;
+      F.red[g][ch] = spl;
     }
-  }
-  // combine the groups: F.red[g] holds the plain sums, F.qraw[g] the stored-basis sums
-  for (int r = 0; r < NGR; ++r) {
-    if (grp == r) {
-#pragma unroll
-      for (int g = 0; g < MAX_G; ++g) {
-        if (g >= G) break;
-        F.qraw[g][ch] = (r == 0 ? 0.f : F.qraw[g][ch]) + srot[g];
-        F.red[g][ch] = (r == 0 ? 0.f : F.red[g][ch]) + spl[g];
-      }
-    }
+    if (kb1 >= nspl) break;
+    __syncthreads();  // the stage is free again
+    kb0 = kb1;
+    kb1 = min(nspl, kb0 + kper);
+    const float *src = part + (int64_t)kb0 * G * PSTRIDE;
+    for (int p = tid; p < (kb1 - kb0) * G * (PSTRIDE / 4); p += DT) cp_async16(stage + 4 * p, src + 4 * p);
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncthreads();
   }
+  __syncthreads();
   // output: (H.acc_rot.kappa + acc_plain) / L, one warp per query head
   for (int g = warp; g < G; g += NW) {
     float v[4];
@@ -934,11 +953,12 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
       for (int e = 0; e < 4; ++e) v[e] *= kKappa();
     }
     const float Lg = F.Ls[g];
+    const float inv = Lg > 0.f ? 1.0f / Lg : 0.f;
     float4 o;
-    o.x = Lg > 0.f ? (v[0] + F.red[g][4 * lane + 0]) / Lg : 0.f;
-    o.y = Lg > 0.f ? (v[1] + F.red[g][4 * lane + 1]) / Lg : 0.f;
-    o.z = Lg > 0.f ? (v[2] + F.red[g][4 * lane + 2]) / Lg : 0.f;
-    o.w = Lg > 0.f ? (v[3] + F.red[g][4 * lane + 3]) / Lg : 0.f;
+    o.x = (v[0] + F.red[g][4 * lane + 0]) * inv;
+    o.y = (v[1] + F.red[g][4 * lane + 1]) * inv;
+    o.z = (v[2] + F.red[g][4 * lane + 2]) * inv;
+    o.w = (v[3] + F.red[g][4 * lane + 3]) * inv;
     *reinterpret_cast<float4 *>(A.out + ((int64_t)s.row * A.hkv * G + head * G + g) * D + 4 * lane) = o;
   }
   if (tid == 0) A.tickets[s.seq * A.hkv + head] = 0u;
@@ -947,6 +967,8 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
 template <int FAM, int BITS>
 cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st) {
   constexpr size_t smem = smem_bytes<FAM, BITS>();
+  static_assert(smem <= 232448, "shared memory per CTA");
+  static_assert((nwarps(FAM, BITS) * warp_area<FAM, BITS>()) / (PSTRIDE * 4) >= MAX_G, "merge stage holds a split");
   static bool attr = false;
   if (!attr) {
     const cudaError_t e = cudaFuncSetAttribute(k_decode<FAM, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
