@@ -25,7 +25,6 @@ namespace {
 constexpr unsigned FULL = 0xffffffffu;
 // warps per CTA (one CTA per SM): 12 where the per-warp stages fit, 8 for 6/8-bit codes
 __host__ __device__ constexpr int nwarps(int fam, int bits) { return (fam != 0 && bits <= 5) ? 12 : 8; }
-constexpr int NWMAX = 12;
 constexpr int CH = 32;       // tokens per chunk (one per lane)
 constexpr int MAXSQ = 48;    // max splits over the quantized prefix per (seq, head)
 constexpr int MAXST = 16;    // max splits over the tail per (seq, head)
@@ -74,14 +73,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Rows 0..7 carry the high int8 limb and rows 8..15 the low limb of a 16-bit fixed-point
 // operand of query head g (Q for Q.K, the softmax weights for P.V); both MMA results of one
 // column combine exactly in int32 as 256*hi + lo.
-
-__device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 // d = a.b + (bias in every element): the accumulator input is one shared register, so no
 // per-MMA reinitialization is needed
@@ -189,10 +180,6 @@ struct VQuad {
   }
 };
 
-__device__ __forceinline__ uint32_t pack_s8(int a, int b, int c, int d) {
-  return (uint32_t)(a & 255) | ((uint32_t)(b & 255) << 8) | ((uint32_t)(c & 255) << 16) | ((uint32_t)(d & 255) << 24);
-}
-
 __device__ __forceinline__ float h2f(const __half *p, int i) { return __half2float(p[i]); }
 
 // 2^x by the MUFU unit (flushes results below 2^-126 to 0: negligible softmax weights)
@@ -239,16 +226,31 @@ struct Stage {
   static constexpr int NST = BITS <= 3 ? 3 : 2;  // stages per warp
 };
 
+// Source cursor of a warp's copies: the K and V sub-pages of the page being copied, looked up
+// in the page table once per page.
+struct PageCursor {
+  int64_t page = -1;
+  const uint8_t *sk = nullptr, *sv = nullptr;
+  __device__ __forceinline__ void seek(const LayerView &L, int seq, int head, int64_t p) {
+    if (p != page) {
+      page = p;
+      sk = subpage_ptr(L, seq, p, head, 0);
+      sv = sk + L.sub_k;
+    }
+  }
+};
+
 // Copies chunk [i0, i0+32) (K and V codes, fp16 scales, and for kvarn the page's channel
 // scales) into the stage `st`, 16 bytes per lane and instruction, as one commit group.
 template <int FAM, int BITS>
-__device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head, int64_t i0, uint8_t *st, int lane) {
+__device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head, int64_t i0, uint8_t *st, int lane,
+                                           PageCursor &pc) {
   using S = Stage<FAM, BITS>;
   const SubLayout lay = sub_layout(FAM, BITS);
-  const int64_t page = i0 / GROUP;
+  pc.seek(L, seq, head, i0 / GROUP);
   const int tip0 = (int)(i0 % GROUP);
-  const uint8_t *sk = subpage_ptr(L, seq, page, head, 0);
-  const uint8_t *sv = subpage_ptr(L, seq, page, head, 1);
+  const uint8_t *sk = pc.sk;
+  const uint8_t *sv = pc.sv;
   constexpr int KP = 32 * BITS;  // 16-byte pieces of K codes (and of V codes)
   constexpr int QP = 4 * BITS;   // pieces per V quad
   const uint8_t *kc = sk + tip0 * 16 * BITS;
@@ -292,26 +294,92 @@ struct ChunkTabs {
 constexpr int kBias = 0x4B400000;       // float bits of 1.5 * 2^23
 constexpr float kBiasF = 12582912.0f;  // an int32 accumulator started at kBias reads as kBiasF + sum
 
-// Issues the first NST - 1 chunks of a warp's range (one commit group each, empty groups past
-// the end), so that their copies overlap the query prologue.
+// Query fragments of one page: the query of head g times the page's K channel scales c
+// (kvarn), in 16-bit fixed point relative to the head's max, split into int8 limbs (hi in
+// rows 0..7, lo in rows 8..15 of the MMA A operand; lane (g, tq) holds channels
+// 32 blk + 8 tq + (0..7)).  sigp undoes the fixed point and the codes' byte position.
+struct QFrag {
+  uint32_t qa[4][4];
+  float sigp;
+  float qs[4];  // qb_1: the query summed over each block
+};
+
 template <int FAM, int BITS>
-__device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq, int head, int64_t a, int64_t c0,
-                                                    int64_t c1, uint8_t *stages, int lane) {
+__device__ __forceinline__ void make_qfrag(QFrag &f, const float (*qrot)[D], const __half *ck, int g, int tq,
+                                           bool hv) {
+  constexpr float SCL = (float)(1 << BITS) / 256.0f / QFIX;
+  float qv[32], amax = 0.f;
+#pragma unroll
+  for (int blk = 0; blk < 4; ++blk) {
+    const float4 q0 = *reinterpret_cast<const float4 *>(&qrot[g][32 * blk + 8 * tq]);
+    const float4 q1 = *reinterpret_cast<const float4 *>(&qrot[g][32 * blk + 8 * tq + 4]);
+    const float qq[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    float cc[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+    if constexpr (FAM == FAM_KVARN) {
+      const uint4 c8 = *reinterpret_cast<const uint4 *>(ck + 32 * blk + 8 * tq);
+      const __half2 *c2 = reinterpret_cast<const __half2 *>(&c8);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 cf = __half22float2(c2[u]);
+        cc[2 * u] = cf.x;
+        cc[2 * u + 1] = cf.y;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float v = hv ? qq[i] * cc[i] : 0.f;
+      qv[blk * 8 + i] = v;
+      amax = fmaxf(amax, fabsf(v));
+    }
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+  const float inv = amax > 0.f ? QFIX * __frcp_rn(amax) : 0.f;
+  f.sigp = amax * SCL;
+  // x * inv rounded to an integer by one FFMA with 1.5 * 2^23 + 128: the float's low bytes
+  // are (qi + 128) mod 2^16, whose byte 1 is the hi limb and byte 0 (with bit 7 flipped) the lo
+#pragma unroll
+  for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = __float_as_uint(fmaf(qv[blk * 8 + 4 * h + i], inv, MAGIC));
+      const uint32_t x = __byte_perm(w[0], w[1], 0x5140), y = __byte_perm(w[2], w[3], 0x5140);
+      f.qa[blk][2 * h] = __byte_perm(x, y, 0x7632);
+      f.qa[blk][2 * h + 1] = __byte_perm(x, y, 0x5410) ^ 0x80808080u;
+    }
+    if constexpr (FAM == FAM_ASYM) {
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum += qv[blk * 8 + i];
+      sum += __shfl_xor_sync(FULL, sum, 1);
+      sum += __shfl_xor_sync(FULL, sum, 2);
+      f.qs[blk] = sum;
+    }
+  }
+}
+
+// Issues the first NST - 1 chunks of a warp's range [c0, c1) (one commit group each, empty
+// groups past the end), so that their copies overlap the query prologue.
+template <int FAM, int BITS>
+__device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq, int head, int64_t a, int c0, int c1,
+                                                    uint8_t *stages, int lane, PageCursor &pc) {
   using S = Stage<FAM, BITS>;
 #pragma unroll
   for (int j = 0; j < S::NST - 1; ++j) {
-    if (j < c1 - c0) copy_chunk<FAM, BITS>(L, seq, head, a + (c0 + j) * CH, stages + j * S::BYTES, lane);
+    if (c0 + j < c1) copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)(c0 + j) * CH, stages + j * S::BYTES, lane, pc);
     cp_async_commit();
   }
 }
 
-// Q.K and P.V of one warp over its chunks [c0, c1) of a quantized split starting at token a
-// (chunks are consecutive, so pages change rarely).  Writes the warp's online-softmax state
-// (m, l and the accumulator in the stored basis) of its heads to shared memory.
+// Q.K and P.V of one warp over its chunks [c0, c1) of a quantized split [a, b) (consecutive, so
+// pages change rarely).  Writes the warp's online-softmax state (m, l and the accumulator in the
+// stored basis) of its heads to shared memory.
 template <int FAM, int BITS>
-__device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
-                                           int64_t c1, int G, const float (*qrot)[D], uint8_t *stages,
-                                           ChunkTabs &T, float *mw, float *lw, float *accw) {
+__device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head, int64_t a, int64_t b, int c0,
+                                           int c1, int G, const float (*qrot)[D], uint8_t *stages, ChunkTabs &T,
+                                           float *mw, float *lw, float *accw, PageCursor &pc) {
   using S = Stage<FAM, BITS>;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -325,69 +393,29 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
   for (int i = 0; i < 32; ++i) acc[i] = 0.f;
   float aoff[4] = {0.f, 0.f, 0.f, 0.f};
   float m_run = -INFINITY, l_run = 0.f;
-  uint32_t qa[4][4];
-  float sigp = 0.f, qs[4] = {0.f, 0.f, 0.f, 0.f};
-  int64_t cur_page = -1;
+  QFrag qf;
+  int cur_page = -1;
 
-  const int nj = (int)(c1 - c0);
-  // the first NST - 1 chunks are already in flight (warp_quant_prefetch)
+  int si = 0;  // stage of chunk c
 #pragma unroll 1
-  for (int j = 0; j < nj; ++j) {
-    const int si = j % S::NST;
-    uint8_t *st = stages + si * S::BYTES;
-    {  // keep NST - 1 chunks in flight: issue chunk j + NST - 1 into the stage read last round
-      const int jn = j + S::NST - 1;
-      if (jn < nj) copy_chunk<FAM, BITS>(L, seq, head, a + (c0 + jn) * CH, stages + (jn % S::NST) * S::BYTES, lane);
+  for (int c = c0; c < c1; ++c) {
+    {  // keep NST - 1 chunks in flight: issue chunk c + NST - 1 into the stage read last round
+      const int cn = c + S::NST - 1;
+      const int sn = si == 0 ? S::NST - 1 : si - 1;
+      if (cn < c1) copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)cn * CH, stages + sn * S::BYTES, lane, pc);
       cp_async_commit();
-    }
-    cp_async_wait<S::NST - 1>();  // chunk j has landed (for this lane's copies)
-    __syncwarp();                 // ... and for every lane's
-    const int64_t i0 = a + (c0 + j) * CH;
-    const int64_t page = i0 / GROUP;
-    const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
-    if (page != cur_page && (FAM == FAM_KVARN || cur_page < 0)) {
-      // query of head g in 16-bit fixed point (two int8 limbs), times the page's K channel
-      // scales c for kvarn; the lane covers channels 32 blk + 8 tq + (0..7)
-      float qv[32], amax = 0.f;
-      const __half *ck = reinterpret_cast<const __half *>(st + S::KCS);
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int ch = 32 * blk + 8 * tq + i;
-          float v = hv ? qrot[g][ch] : 0.f;
-          if (FAM == FAM_KVARN) v *= h2f(ck, ch);
-          qv[blk * 8 + i] = v;
-          amax = fmaxf(amax, fabsf(v));
-        }
-      amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
-      const float inv = amax > 0.f ? QFIX * __frcp_rn(amax) : 0.f;
-      sigp = amax * SCL;
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        int hi[8], lo[8];
-        float sum = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int qi = __float2int_rn(qv[blk * 8 + i] * inv);
-          hi[i] = (qi + 128) >> 8;
-          lo[i] = qi - (hi[i] << 8);
-          sum += qv[blk * 8 + i];
-        }
-        qa[blk][0] = pack_s8(hi[0], hi[1], hi[2], hi[3]);
-        qa[blk][1] = pack_s8(lo[0], lo[1], lo[2], lo[3]);
-        qa[blk][2] = pack_s8(hi[4], hi[5], hi[6], hi[7]);
-        qa[blk][3] = pack_s8(lo[4], lo[5], lo[6], lo[7]);
-        if (FAM == FAM_ASYM) {
-          sum += __shfl_xor_sync(FULL, sum, 1);
-          sum += __shfl_xor_sync(FULL, sum, 2);
-          qs[blk] = sum;
-        }
+      cp_async_wait<S::NST - 1>();  // chunk c has landed (for this lane's copies)
+      __syncwarp();                 // ... and for every lane's
+      uint8_t *st = stages + si * S::BYTES;
+      si = si + 1 == S::NST ? 0 : si + 1;
+      const int64_t i0 = a + (int64_t)c * CH;
+      const int page = (int)(i0 / GROUP);
+      const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
+      if (page != cur_page && (FAM == FAM_KVARN || cur_page < 0)) {
+        make_qfrag<FAM, BITS>(qf, qrot, reinterpret_cast<const __half *>(st + S::KCS), g, tq, hv);
+        cur_page = page;
       }
-    }
-    cur_page = page;
-
+      const float sigp = qf.sigp;
     // ---- scale tables: lane = token of the chunk; rows past the end of the context may hold
     //      stale bytes and get zero scales, so they never reach a sum
     float scl[4];
@@ -455,7 +483,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
         uint32_t b0, b1;
         kt.frag(blk, tq, b0, b1);
         int c[4];
-        mma_s8_bias(c, qa[blk], b0, b1, kBias);
+        mma_s8_bias(c, qf.qa[blk], b0, b1, kBias);
         const float h0 = __int_as_float(c[0]) - kBiasF, h1 = __int_as_float(c[1]) - kBiasF;
         const float l0 = __int_as_float(c[2]) - kBiasF, l1 = __int_as_float(c[3]) - kBiasF;
         x0 = fmaf(d0[blk], fmaf(256.f, h0, l0), x0);
@@ -465,8 +493,8 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       if (FAM == FAM_ASYM) {
         const float4 mA = *reinterpret_cast<const float4 *>(&T.km[t0][0]);
         const float4 mB = *reinterpret_cast<const float4 *>(&T.km[t0 + 1][0]);
-        s0 = fmaf(mA.x, qs[0], fmaf(mA.y, qs[1], fmaf(mA.z, qs[2], fmaf(mA.w, qs[3], s0))));
-        s1 = fmaf(mB.x, qs[0], fmaf(mB.y, qs[1], fmaf(mB.z, qs[2], fmaf(mB.w, qs[3], s1))));
+        s0 = fmaf(mA.x, qf.qs[0], fmaf(mA.y, qf.qs[1], fmaf(mA.z, qf.qs[2], fmaf(mA.w, qf.qs[3], s0))));
+        s1 = fmaf(mB.x, qf.qs[0], fmaf(mB.y, qf.qs[1], fmaf(mB.z, qf.qs[2], fmaf(mB.w, qf.qs[3], s1))));
       }
       sc[2 * r] = t0 < nvalid ? s0 : -INFINITY;
       sc[2 * r + 1] = t0 + 1 < nvalid ? s1 : -INFINITY;
@@ -486,7 +514,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       p[k] = sc[k] == -INFINITY ? 0.f : exp2_fast(sc[k] - mn);
       psum += p[k];
     }
-    if (alpha != 1.f) {
+    if (__any_sync(FULL, alpha != 1.f)) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc[i] *= alpha;
 #pragma unroll
@@ -555,7 +583,8 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       }
     }
 
-    __syncwarp();  // every lane is done with stage si before it is refilled next round
+    __syncwarp();  // every lane is done with this stage before it is refilled next round
+    }
   }
   cp_async_wait<0>();
   __syncwarp();
@@ -729,7 +758,6 @@ template <int NW>
 struct SmemFixed {
   float qraw[MAX_G][D];
   float qrot[MAX_G][D];
-  float pst[NW][CH][MAX_G];
   float mw[NW][MAX_G], lw[NW][MAX_G];
   float fw[MAXSPL][MAX_G];   // weight of each warp (CTA combine) / split (merge)
   float fm[MAXSPL][MAX_G];   // merge: m and l of the splits whose records are not staged
@@ -751,10 +779,15 @@ __host__ __device__ constexpr int warp_area() {
   }
 }
 
+// [SmemFixed][warp areas]
+template <int FAM, int BITS>
+__host__ __device__ constexpr size_t smem_fixed_bytes() {
+  return ((sizeof(SmemFixed<nwarps(FAM, BITS)>) + 127) / 128) * 128;
+}
+
 template <int FAM, int BITS>
 __host__ __device__ constexpr size_t smem_bytes() {
-  constexpr int NW = nwarps(FAM, BITS);
-  return ((sizeof(SmemFixed<NW>) + 127) / 128) * 128 + (size_t)NW * warp_area<FAM, BITS>();
+  return smem_fixed_bytes<FAM, BITS>() + (size_t)nwarps(FAM, BITS) * warp_area<FAM, BITS>();
 }
 
 template <int FAM, int BITS>
@@ -762,7 +795,7 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
   constexpr int NW = nwarps(FAM, BITS), DT = 32 * NW;
   extern __shared__ __align__(128) uint8_t smem[];
   SmemFixed<NW> &F = *reinterpret_cast<SmemFixed<NW> *>(smem);
-  uint8_t *warp_mem = smem + ((sizeof(SmemFixed<NW>) + 127) / 128) * 128;
+  uint8_t *warp_mem = smem + smem_fixed_bytes<FAM, BITS>();
   constexpr int WA = warp_area<FAM, BITS>();
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -785,12 +818,13 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
     b = min(a + (int64_t)s.cps_t * CH, s.n);
   }
   nch = b > a ? (b - a + CH - 1) / CH : 0;
-  // contiguous chunk range of this warp
+  // a contiguous chunk range per warp
   const int64_t per = (nch + NW - 1) / NW;
   const int64_t c0 = min((int64_t)warp * per, nch), c1 = min(c0 + per, nch);
 
+  PageCursor pc;
   if constexpr (FAM != FAM_BF16) {
-    if (!tail) warp_quant_prefetch<FAM, BITS>(L, s.seq, head, a, c0, c1, warp_mem + (size_t)warp * WA, lane);
+    if (!tail) warp_quant_prefetch<FAM, BITS>(L, s.seq, head, a, (int)c0, (int)c1, warp_mem + (size_t)warp * WA, lane, pc);
   }
   // query rows of this KV head, pre-scaled by softmax_scale * log2(e); heads >= G are 0
   for (int idx = tid; idx < MAX_G * D; idx += DT) {
@@ -818,19 +852,22 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
   __syncthreads();
 
   float *accw = reinterpret_cast<float *>(warp_mem + (size_t)warp * WA);  // [MAX_G][D] after the chunks
+  // BF16 warps: softmax weights of a chunk, after the accumulator in the warp area
+  float(*pst)[MAX_G] = reinterpret_cast<float(*)[MAX_G]>(warp_mem + (size_t)warp * WA + MAX_G * D * 4);
+  static_assert(WA >= MAX_G * D * 4 + CH * MAX_G * 4, "warp area holds accumulator and weights");
   if constexpr (FAM != FAM_BF16) {
     if (!tail) {
-      warp_quant<FAM, BITS>(L, s.seq, head, a, b, c0, c1, G, F.qrot, warp_mem + (size_t)warp * WA, F.tabs[warp],
-                            F.mw[warp], F.lw[warp], accw);
+      warp_quant<FAM, BITS>(L, s.seq, head, a, b, (int)c0, (int)c1, G, F.qrot, warp_mem + (size_t)warp * WA,
+                            F.tabs[warp], F.mw[warp], F.lw[warp], accw, pc);
     } else {
       for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
       __syncwarp();
-      warp_bf16(L, s.seq, head, a, b, c0, c1, G, F.qraw, F.pst[warp], F.mw[warp], F.lw[warp], accw);
+      warp_bf16(L, s.seq, head, a, b, c0, c1, G, F.qraw, pst, F.mw[warp], F.lw[warp], accw);
     }
   } else {
     for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
     __syncwarp();
-    warp_bf16(L, s.seq, head, a, b, c0, c1, G, F.qraw, F.pst[warp], F.mw[warp], F.lw[warp], accw);
+    warp_bf16(L, s.seq, head, a, b, c0, c1, G, F.qraw, pst, F.mw[warp], F.lw[warp], accw);
   }
   __syncthreads();
 
