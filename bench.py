@@ -357,11 +357,145 @@ def run_type_sweep(args, kvq, torch, synth, cfg):
     return out
 
 
+def graph_time_us(torch, fn, reps=10):
+    """Mean duration in microseconds of one replay of a CUDA graph of fn()."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def run_formats(args, kvq, torch, synth):
+    """Plain block formats at context 16384 with tails 0 / 1024 / 2048 (8 KV heads, 32 query
+    heads): decode GB/s, cycling enough layer caches that every decode reads from HBM."""
+    calc = LibCalc(kvq)
+    cfg = synth.config1()
+    n, hkv, hq = cfg["n"], cfg["hkv"], cfg["hq"]
+    kt = dev_bf16(torch, synth.token_major(cfg["k"]))
+    vt = dev_bf16(torch, synth.token_major(cfg["v"]))
+    qdev = torch.from_numpy(cfg["q"][0, 0]).cuda()[None]
+    o = torch.empty_like(qdev)
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    out = {}
+    for t in cfg["types"]:
+        for tail in cfg["tails"]:
+            b = decode_bytes(calc, t, n, tail, hkv, hq)
+            L = max(2, math.ceil(4 * l2 / b))
+            cache = kvq.KVCache(n_layers=L, n_seqs=1, n_kv_heads=hkv, max_ctx=n, type_k=t, type_v=t, tail=tail)
+            for l in range(L):
+                cache.append(l, [0], [n], kt, vt)
+            cache.workspace(1, hq)
+
+            def fn():
+                for i in range(4 * L):
+                    cache.decode(i % L, [0], qdev, out=o)
+
+            us = graph_time_us(torch, fn) / (4 * L)
+            out[f"{t}/T{tail}"] = {"decode_us": round(us, 2), "GB_per_s": round(b / us / 1e3, 1), "bytes": int(b),
+                                   "layers_cycled": L}
+            assert cache.status() == 0
+            del cache
+            torch.cuda.empty_cache()
+    return {"workload": f"context {n}, {hkv} KV heads x 128, {hq} query heads, batch 1, tails {cfg['tails']}",
+            "per_format": out}
+
+
+def run_page1_shape(args, kvq, torch, synth):
+    """64 layers x 8 KV heads x 128, 64 query heads, context 240000: one decode over all 64
+    layers (one CUDA graph), kvarn2 and q4_0 with a 1024-token tail, and all-BF16.  The
+    seeded data of layer 0 is appended to every layer (the kernels' timing does not depend
+    on the values)."""
+    calc = LibCalc(kvq)
+    cfg = synth.config4_layer(0)
+    n, hkv, hq, tail = cfg["n"], cfg["hkv"], cfg["hq"], cfg["tail"]
+    NL = 64
+    kt = dev_bf16(torch, synth.token_major(cfg["k"]))
+    vt = dev_bf16(torch, synth.token_major(cfg["v"]))
+    qdev = torch.from_numpy(cfg["q"][0, 0]).cuda()[None]
+    o = torch.empty((NL, 1, hq, D), dtype=torch.float32, device="cuda")
+    out = {}
+    for t in cfg["types"]:
+        tl = tail if t != "bf16" else 0
+        cache = kvq.KVCache(n_layers=NL, n_seqs=1, n_kv_heads=hkv, max_ctx=n, type_k=t, type_v=t, tail=tl)
+        for l in range(NL):
+            cache.append(l, [0], [n], kt, vt)
+        cache.workspace(1, hq)
+
+        def fn():
+            for l in range(NL):
+                cache.decode(l, [0], qdev, out=o[l])
+
+        us = graph_time_us(torch, fn, reps=3)
+        b = NL * decode_bytes(calc, t, n, tl, hkv, hq)
+        out[t] = {"decode_64_layers_ms": round(us / 1e3, 3), "GB_per_s": round(b / us / 1e3, 1), "bytes": int(b),
+                  "cache_bytes": int(cache.nbytes)}
+        assert cache.status() == 0
+        del cache
+        torch.cuda.empty_cache()
+    return {"workload": f"{NL} layers, context {n}, {hkv} KV heads x 128, {hq} query heads, batch 1, "
+                        f"tail {tail} (quantized types); layer 0's seeded data in every layer", "per_type": out}
+
+
+def run_quality(args, kvq, torch, synth):
+    """Side report (not a target): attention KL(P_bf16 || P_q) and the relative L2 error of the
+    attention output of a quantized cache against the BF16 cache of the same data, for every
+    type and the tail sizes 0..2048 (context 16384, 8 KV heads, 32 query heads, 4 query
+    draws).  The cache is read back through kvq_dequant (original basis); the attention
+    itself is plain fp32 torch, outside the product path."""
+    cfg = synth.config1()
+    n, hkv, hq = cfg["n"], cfg["hkv"], cfg["hq"]
+    G = hq // hkv
+    rng = np.random.default_rng(11)
+    q = torch.from_numpy(rng.standard_normal((4, hq, D)).astype(np.float32)).cuda()
+    kt = dev_bf16(torch, synth.token_major(cfg["k"]))
+    vt = dev_bf16(torch, synth.token_major(cfg["v"]))
+
+    def attend(kf, vf):  # kf, vf: [n, hkv, D] fp32 -> probabilities [4, hq, n], out [4, hq, D]
+        kk = kf.permute(1, 0, 2).repeat_interleave(G, 0)  # [hq, n, D]
+        vv = vf.permute(1, 0, 2).repeat_interleave(G, 0)
+        s = torch.einsum("bhd,hnd->bhn", q, kk) / math.sqrt(D)
+        p = torch.softmax(s, -1)
+        return p, torch.einsum("bhn,hnd->bhd", p, vv)
+
+    p0, o0 = attend(kt.float(), vt.float())
+    lp0 = torch.log(p0.clamp_min(1e-38))
+    types = ["q2_0", "q3_0", "q4_0", "q5_0", "q6_0", "q8_0", "q4_1", "q2_1", "q3_1", "q5_1", "q6_1",
+             "kvarn2", "kvarn3", "kvarn4", "kvarn5", "kvarn6", "kvarn8"]
+    out = {}
+    for t in types:
+        row = {}
+        for tail in (0, 256, 512, 1024, 2048):
+            cache = kvq.KVCache(n_layers=1, n_seqs=1, n_kv_heads=hkv, max_ctx=n, type_k=t, type_v=t, tail=tail)
+            cache.append(0, [0], [n], kt, vt)
+            kf = cache.dequant(0, 0, 0, 0, n)
+            vf = cache.dequant(0, 0, 1, 0, n)
+            p1, o1 = attend(kf, vf)
+            kl = (p0 * (lp0 - torch.log(p1.clamp_min(1e-38)))).sum(-1)  # [4, hq]
+            rel = (o1 - o0).norm(dim=-1) / o0.norm(dim=-1)
+            row[f"T{tail}"] = {"kl_mean": float(kl.mean()), "kl_median": float(kl.median()),
+                               "out_rel_l2_mean": float(rel.mean())}
+            del cache
+        out[t] = row
+    return {"workload": f"context {n}, {hkv} KV heads, {hq} query heads, 4 query draws (seed 11), data as the "
+                        f"formats workload", "per_type": out}
+
+
 def run_append(args, kvq, torch, synth):
     """Batched prefill-append: 16 sequences built to L_i ~ U[4096, 32768], then one timed
-    append of 4096 tokens per sequence (kvarn4, tail 1024)."""
-    cfg = synth.config3(steps=0)
-    hkv, tail = cfg["hkv"], cfg["tail"]
+    append of 4096 tokens per sequence (kvarn4, tail 1024), then 64 batched decode steps
+    (one token appended to every sequence, then decode of all 16)."""
+    NSTEP = 64
+    cfg = synth.config3(steps=NSTEP)
+    hkv, hq, tail = cfg["hkv"], cfg["hq"], cfg["tail"]
     Ls = cfg["lengths"]
     S = len(Ls)
     cache = kvq.KVCache(n_layers=1, n_seqs=S, n_kv_heads=hkv, max_ctx=max(Ls) + cfg["prefill"] + 64,
@@ -384,6 +518,34 @@ def run_append(args, kvq, torch, synth):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     assert cache.status() == 0
+
+    # batched decode steps: append one token per sequence, then decode all of them
+    calc = LibCalc(kvq)
+    qd = torch.from_numpy(cfg["q"]).cuda()  # [steps, S, hq, 128]
+    od = torch.empty((S, hq, D), dtype=torch.float32, device="cuda")
+    cache.workspace(S, hq)
+    ksteps = torch.stack([torch.cat([k[l + P + j:l + P + j + 1] for k, l in zip(ks, Ls)]) for j in range(NSTEP)])
+    vsteps = torch.stack([torch.cat([v[l + P + j:l + P + j + 1] for v, l in zip(vs, Ls)]) for j in range(NSTEP)])
+    gs = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gs):
+        for j in range(NSTEP):
+            cache.append(0, list(range(S)), [1] * S, ksteps[j], vsteps[j])
+            cache.decode(0, list(range(S)), qd[j], out=od)
+    e0.record()
+    gs.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    step_ms = e0.elapsed_time(e1) / NSTEP
+    assert cache.status() == 0
+    ctx_end = [l + P + NSTEP for l in Ls]
+    dec_b = sum(decode_bytes(calc, "kvarn4", c, tail, hkv, hq) for c in ctx_end)
+    dec_us = graph_time_us(torch, lambda: cache.decode(0, list(range(S)), qd[0], out=od))
+    batched = {"steps": NSTEP, "ms_per_step": round(step_ms, 4),
+               "step_GB_per_s": round(dec_b / (step_ms * 1e-3) / 1e9, 1),
+               "decode_us": round(dec_us, 2), "decode_GB_per_s": round(dec_b / dec_us / 1e3, 1),
+               "decode_bytes": int(dec_b),
+               "workload": f"{S} sequences at {min(ctx_end)}..{max(ctx_end)} tokens, kvarn4, tail {tail}, "
+                           f"{hkv} KV heads, {hq} query heads; step = append 1 token to each + decode all"}
     # algorithmic bytes: new rows in, the old tail + open-group rows re-read, quantized
     # tokens and the new tail out (per stream)
     tb = 75.0
@@ -396,7 +558,7 @@ def run_append(args, kvq, torch, synth):
     return {"metric": "append Mtok/s", "value": round(S * P / (ms * 1e-3) / 1e6, 2), "unit": "Mtok/s",
             "ms": round(ms, 4), "GB_per_s": round(moved / (ms * 1e-3) / 1e9, 1), "bytes": int(moved),
             "workload": f"{S} sequences, lengths {min(Ls)}..{max(Ls)}, +{P} tokens each in one call, kvarn4, "
-                        f"tail {tail}, 8 KV heads x 128"}
+                        f"tail {tail}, 8 KV heads x 128", "batched_decode": batched}
 
 
 # ---------------------------------------------------------------------------------------
@@ -432,29 +594,41 @@ def traffic_for(kernel, type_):
 # ---------------------------------------------------------------------------------------
 # the CPU oracle
 
-def oracle_decode_sample(cfg, type_, heads, n):
-    """Times the oracle's decode (stream state rebuilt from the BF16 history, fp64
-    dequant + attention) for `heads` KV heads of one step at context n."""
+def _oracle_head_job(job):
+    """One KV head's decode by the oracle (runs in a spawned worker); returns seconds."""
     import oracle
 
-    G = cfg["hq"] // cfg["hkv"]
-    q = cfg["q"][0, 0]
+    type_, k, v, tail, q = job
     t0 = time.perf_counter()
-    for h in heads:
-        oracle.decode_head(type_, type_, cfg["k"][h, :n], cfg["v"][h, :n], cfg["tail"], q[h * G:(h + 1) * G])
+    oracle.decode_head(type_, type_, k, v, tail, q)
     return time.perf_counter() - t0
 
 
 def cpu_baseline(cfg, type_):
+    """The oracle on the host cores: one decode step at 64k (all KV heads), one head per
+    worker process (spawned, so no worker inherits a CUDA context)."""
+    import multiprocessing as mp
+
     import oracle as calc
 
-    n = cfg["n"]
-    heads = [0, 1, 2, 3]
-    dt = oracle_decode_sample(cfg, type_, heads, n)
-    b = decode_bytes(calc, type_, n, cfg["tail"], len(heads), len(heads) * cfg["hq"] // cfg["hkv"])
-    return {"value": round(b / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"one decode step of 1 of {cfg['hkv']} KV heads at context {n} ({type_}), "
-                      f"{dt:.1f} s single-threaded; the oracle rebuilds the stream state from BF16 each call"}
+    n, hkv = cfg["n"], cfg["hkv"]
+    G = cfg["hq"] // hkv
+    q = cfg["q"][0, 0]
+    cores = len(os.sched_getaffinity(0))
+    nproc = max(1, min(cores, hkv))
+    jobs = [(type_, cfg["k"][h, :n], cfg["v"][h, :n], cfg["tail"], q[h * G:(h + 1) * G]) for h in range(hkv)]
+    with mp.get_context("spawn").Pool(nproc) as pool:
+        pool.map(_oracle_head_job, jobs[:nproc])  # start the workers (and load the oracle) untimed
+        t0 = time.perf_counter()
+        per_head = pool.map(_oracle_head_job, jobs)
+        wall = time.perf_counter() - t0
+    b = decode_bytes(calc, type_, n, cfg["tail"], hkv, cfg["hq"])
+    single = b / sum(per_head) / 1e9
+    return {"value": round(b / wall / 1e9, 5), "unit": "GB/s", "cores": nproc, "kind": "oracle",
+            "single_thread_value": round(single, 5),
+            "sample": f"one decode step at context {n} ({type_}, {hkv} KV heads, {cfg['hq']} query heads), one KV "
+                      f"head per worker process on {nproc} of {cores} host cores, {wall:.1f} s wall, "
+                      f"{sum(per_head):.1f} s CPU; the oracle rebuilds each stream's state from BF16 in the call"}
 
 
 def run_reference(args, ws, rank):
@@ -515,6 +689,12 @@ def main():
         result["per_type_decode_64k"] = run_type_sweep(args, kvq, torch, synth, cfg)
         torch.cuda.empty_cache()
         result["append"] = run_append(args, kvq, torch, synth)
+        torch.cuda.empty_cache()
+        result["formats_16k"] = run_formats(args, kvq, torch, synth)
+        torch.cuda.empty_cache()
+        result["page1_shape_240k"] = run_page1_shape(args, kvq, torch, synth)
+        torch.cuda.empty_cache()
+        result["quality"] = run_quality(args, kvq, torch, synth)
     if rank == 0 and ws == 1:
         result["cpu_baseline"] = cpu_baseline(cfg, args.type)
     elif rank == 0:
