@@ -217,6 +217,58 @@ int kvq_workspace_bytes(const kvq_cache *c, int32_t n_seqs, int32_t n_q_heads, s
   return KVQ_OK;
 }
 
+int kvq_append_decode(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,
+                      const int32_t *n_new, const void *k_bf16, const void *v_bf16, int32_t n_q_heads,
+                      const float *q, float softmax_scale, float *out, void *workspace, size_t ws_bytes,
+                      kvq_stream_t stream) {
+  // every argument is checked before anything is launched, so a failed call changes nothing
+  if (!c || layer < 0 || layer >= c->p.n_layers || n_seqs < 0) return KVQ_E_INVAL;
+  if (n_seqs == 0) return KVQ_OK;
+  if (!seq_ids || !n_new || !q || !out || !workspace || n_q_heads < 1) return KVQ_E_INVAL;
+  if (n_q_heads % c->p.n_kv_heads) return KVQ_E_INVAL;
+  if (n_q_heads / c->p.n_kv_heads > MAX_G) return KVQ_E_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_E_ALIGN;
+  if (ws_bytes < decode_workspace_bytes(c, n_seqs, n_q_heads)) return KVQ_E_SIZE;
+  std::vector<char> seen(c->p.n_seqs, 0);
+  std::vector<AppendSeq> app;
+  std::vector<DecodeSeq> dec;
+  int64_t rows = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int s = seq_ids[i];
+    if (s < 0 || s >= c->p.n_seqs || seen[s] || n_new[i] < 0) return KVQ_E_INVAL;
+    seen[s] = 1;
+    const int64_t n0 = c->len[(size_t)layer * c->p.n_seqs + s];
+    if (n0 + n_new[i] > c->p.max_ctx) return KVQ_E_CAPACITY;
+    if (n_new[i] > 0) app.push_back({s, n_new[i], n0, rows});
+    rows += n_new[i];
+    const int64_t n1 = n0 + n_new[i];
+    DecodeSeq d{s, i, n1, quantized_len(c, n1)};
+    if (n_new[i] > 0) {
+      // what this append rewrites: the quantized tokens from the first group (kvarn) or token
+      // (q types) it touches, and the ring rows of the new tokens
+      const int64_t Q0 = quantized_len(c, n0);
+      d.dq = c->fam_k == FAM_KVARN ? (Q0 / GROUP) * GROUP : Q0;
+      d.dt = n0;
+    }
+    dec.push_back(d);
+  }
+  if (rows > 0 && (!k_bf16 || !v_bf16)) return KVQ_E_INVAL;
+  if (rows > 0 && (!aligned16(k_bf16) || !aligned16(v_bf16))) return KVQ_E_ALIGN;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  AppendInfo info;
+  if (rows > 0) {
+    const int rc = launch_append(c, layer, app, k_bf16, v_bf16, st, &info);
+    if (rc) return rc;
+    for (const AppendSeq &a : app) c->len[(size_t)layer * c->p.n_seqs + a.seq] = a.n0 + a.n_new;
+  }
+  // the decode overlaps the append's last kernel; when that kernel is a small spill it keeps
+  // its SMs, so the decode plans for the others
+  const bool pdl = info.launches > 0;
+  const int budget = info.last_ctas > 0 && info.last_ctas <= c->num_sms / 4 ? c->num_sms - info.last_ctas : 0;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
+  return launch_decode(c, layer, dec, n_q_heads, q, scale, out, workspace, ws_bytes, st, budget, pdl);
+}
+
 int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,
                     int32_t n_q_heads, const float *q, float softmax_scale, float *out, void *workspace,
                     size_t ws_bytes, kvq_stream_t stream) {

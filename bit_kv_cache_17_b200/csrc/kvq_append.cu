@@ -10,7 +10,12 @@
 //     group touched by the append is rebuilt from its BF16 rows (ring or new input):
 //     Walsh-Hadamard rotation -> Sinkhorn balancing -> symmetric block quantization;
 //  2. the new tokens that stay 16-bit are copied into the BF16 ring.
-// Step 1 reads ring rows that step 2 may overwrite, so step 2 is launched after it.
+// Step 1 reads ring rows that step 2 may overwrite, so step 2 is launched after it, unless
+// no ring slot that step 2 writes can hold a row that step 1 reads (the span from the first
+// row read to the last row written fits in the ring, as for one-token appends to a kvarn
+// cache): then the spill kernel writes the new rows itself and one launch does both.
+// Every kernel here signals its dependents as it starts (griddepcontrol.launch_dependents),
+// so that a decode launched with programmatic stream serialization may overlap it.
 #include <cuda_runtime.h>
 
 #include "kvq_internal.h"
@@ -28,7 +33,10 @@ struct SeqWork {
   int64_t in_off;    // first input row of this sequence
   int64_t a, b;      // kernel-specific range
   int64_t item0;     // first work item of this sequence
+  int64_t tw;        // k_spill_kvarn: new rows [tw, n1) go to the ring in this launch
 };
+
+__device__ __forceinline__ void signal_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 struct Work {
   int32_t n;
@@ -199,6 +207,7 @@ template <int FAM, int BITS, int WHICH>
 __global__ void __launch_bounds__(256) k_spill_qb(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in) {
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  signal_dependents();
   if (item >= W.total) return;
   const SeqWork &s = W.s[find_seq(W, item)];
   const int64_t local = item - s.item0;
@@ -242,6 +251,48 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   return d;
 }
 
+// Packed fp32 pairs in one 64-bit register (sm_100 f32x2 arithmetic): each lane is rounded
+// once, exactly as the scalar operation with the same operands.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(f32x2 v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// rint(RN(y / d)) for the codes of one block, by the reciprocal.  With rd = RN(1/d) and
+// q = RN(y * rd), |q - RN(y / d)| <= 2^-15.4 for |q| <= 128 (two roundings of 2^-24 relative
+// each, plus the quotient's own).  q + 1.5 * 2^23 rounds q to the nearest integer, ties to
+// even, and its low bits are that integer in two's complement (the code, before masking);
+// subtracting the constant back gives r = rint(q) exactly and t = q - r exactly.  Where
+// |t| <= 0.5 - 2^-13 no half-integer lies between q and RN(y / d), so both round to r; where
+// any |t| of the block is larger, the caller takes the exact quotients instead.
+constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
+constexpr float kTieBound = 0.4998779296875f;  // 0.5 - 2^-13
+
 // Thread-per-token quantization of a balanced group (see k_spill_kvarn, step 4).  The block
 // loop is kept rolled: the kernel is long straight-line code executed once per CTA, so its
 // instruction footprint, not its arithmetic, sets the pace.
@@ -252,44 +303,60 @@ __device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const Sub
   uint8_t *img = reinterpret_cast<uint8_t *>(S.img);
   if (tid < ng) {
     const float rti = S.rt[tid];
+    const float *xr = &S.X[tid * XS];
     uint32_t dlo = 0u, dhi = 0u;
 #pragma unroll 1
     for (int blk = 0; blk < 4; ++blk) {
-      float y[32];
+      // y = (x * rc_j) * rt_i, two roundings, on channel pairs
+      f32x2 yp[16];
       float amax = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        y[e] = __fmul_rn(__fmul_rn(S.X[tid * XS + 32 * blk + e], S.rc[32 * blk + e]), rti);
-        amax = fmaxf(amax, fabsf(y[e]));
+      for (int i = 0; i < 16; ++i) {
+        const f32x2 rcp = *reinterpret_cast<const f32x2 *>(&S.rc[32 * blk + 2 * i]);
+        yp[i] = mul2(mul2(pk2(xr[32 * blk + 2 * i], xr[32 * blk + 2 * i + 1]), rcp), pk2(rti, rti));
+        float y0, y1;
+        upk2(yp[i], y0, y1);
+        amax = max3(amax, fabsf(y0), fabsf(y1));
       }
       const __half dh = sat_half(__fdiv_rn(amax, (float)QMAX));
       const float df = __half2float(dh);
-      const float rd = df != 0.0f ? __frcp_rn(df) : 0.0f;
+      const unsigned short dbits = __half_as_ushort(dh) & 0x7fffu;
       const uint32_t dv = (uint32_t)__half_as_ushort(dh) << (16 * (blk & 1));
       if (blk < 2)
         dlo |= dv;
       else
         dhi |= dv;
-      // rint(RN(y/d)) by the reciprocal; the exact quotient only where a value sits within 4 ulp
-      // of a half-integer (checked once for the block)
-      float r[32];
-      bool tie = false;
+      uint32_t f[32];  // low BITS bits: the code in two's complement
+      // a normal, unsaturated d keeps |y / d| <= QMAX (1 + 2^-11): no clamp needed
+      const bool plain = dbits >= 0x0400u && dbits != 0x7bffu;
+      bool tie = !plain;
+      if (plain) {
+        const float rd = __frcp_rn(df);
+        const f32x2 rd2 = pk2(rd, rd), mg = pk2(kRintMagic, kRintMagic);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float q = __fmul_rn(y[e], rd);
-        r[e] = rintf(q);
-        const float tol = fmaxf(fabsf(q), 1.0f) * 9.5367431640625e-07f;
-        tie |= fabsf(fabsf(__fsub_rn(q, r[e])) - 0.5f) <= tol;
+        for (int i = 0; i < 16; ++i) {
+          const f32x2 q = mul2(yp[i], rd2);
+          const f32x2 m = add2(q, mg);
+          float t0, t1, m0, m1;
+          upk2(sub2(q, sub2(m, mg)), t0, t1);
+          upk2(m, m0, m1);
+          tie |= fabsf(t0) > kTieBound;
+          tie |= fabsf(t1) > kTieBound;
+          f[2 * i] = __float_as_uint(m0);
+          f[2 * i + 1] = __float_as_uint(m1);
+        }
       }
-      if (tie) {
+      if (tie) {  // exact quotients (rare), clamped; d = 0 gives zero codes
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = rintf(__fdiv_rn(y[e], df));
-      }
-      uint32_t f[32];
+        for (int i = 0; i < 16; ++i) {
+          float y[2];
+          upk2(yp[i], y[0], y[1]);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float rr = df != 0.0f ? fminf(fmaxf(r[e], (float)QMIN), (float)QMAX) : 0.0f;
-        f[e] = (uint32_t)(int)rr & ((1u << BITS) - 1u);
+          for (int e = 0; e < 2; ++e) {
+            const float rr = df != 0.0f ? fminf(fmaxf(rintf(__fdiv_rn(y[e], df)), (float)QMIN), (float)QMAX) : 0.0f;
+            f[2 * i + e] = (uint32_t)(int)rr;
+          }
+        }
       }
 #pragma unroll
       for (int pl = 0; pl < 2; ++pl) {
@@ -369,6 +436,16 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
   const int ng = (int)((Q1 - g0) < GROUP ? (Q1 - g0) : GROUP);
   const SubLayout lay = sub_layout(FAM_KVARN, BITS);
   uint8_t *sub = subpage_ptr(L, s.seq, g, head, which);
+  signal_dependents();
+
+  // 0. fused ring write: the CTA of the stream's last group copies the new rows that stay
+  //    16-bit (16 threads per 256-byte row); no row it writes shares a slot with a row read here
+  if (g0 + GROUP >= Q1) {
+    for (int64_t p = s.tw + tid / 16; p < s.n1; p += KV_THREADS / 16) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(in + ((s.in_off + (p - s.n0)) * L.hkv + head) * D);
+      reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, which, p))[tid & 15] = src[tid & 15];
+    }
+  }
 
   // 1. each thread rotates one row in registers: BF16 -> fp32, butterfly h = 1..64, x kappa
   if (tid < ng) {
@@ -384,18 +461,35 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         r[8 * j8 + 2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
       }
     }
+    // stage h = 1 on scalars; stages h = 2..64 pair channels (2i, 2i+1) with (2i+h, 2i+1+h),
+    // two butterflies per packed add / sub
 #pragma unroll
-    for (int h = 1; h < D; h <<= 1) {
+    for (int j = 0; j < D; j += 2) {
+      const float x = r[j], y = r[j + 1];
+      r[j] = __fadd_rn(x, y);
+      r[j + 1] = __fsub_rn(x, y);
+    }
+    f32x2 rp[D / 2];
 #pragma unroll
-      for (int j = 0; j < D; ++j) {
-        if (j & h) continue;
-        const float x = r[j], y = r[j + h];
-        r[j] = __fadd_rn(x, y);
-        r[j + h] = __fsub_rn(x, y);
+    for (int i = 0; i < D / 2; ++i) rp[i] = pk2(r[2 * i], r[2 * i + 1]);
+#pragma unroll
+    for (int hp = 1; hp < D / 2; hp <<= 1) {
+#pragma unroll
+      for (int i = 0; i < D / 2; ++i) {
+        if (i & hp) continue;
+        const f32x2 a = rp[i], b = rp[i + hp];
+        rp[i] = add2(a, b);
+        rp[i + hp] = sub2(a, b);
       }
     }
+    const f32x2 kk = pk2(kKappa(), kKappa());
 #pragma unroll
-    for (int j = 0; j < D; ++j) S.X[tid * XS + j] = __fmul_rn(r[j], kKappa());
+    for (int i = 0; i < D / 2; ++i) {
+      float a, b;
+      upk2(mul2(rp[i], kk), a, b);
+      S.X[tid * XS + 2 * i] = a;
+      S.X[tid * XS + 2 * i + 1] = b;
+    }
   }
   if (tid < GROUP) S.uS[tid & 31][tid >> 5] = 1.0f;  // first iteration: t = 1
   __syncthreads();
@@ -542,6 +636,7 @@ __global__ void __launch_bounds__(256) k_tail_write(LayerView L, Work W, const _
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   int64_t item = t >> 4;
   const int part = (int)(t & 15);
+  signal_dependents();
   if (item >= W.total) return;
   int which = W.which;
   if (which == 2) {  // K and V in one launch: the first half of the items is K
@@ -604,7 +699,10 @@ cudaError_t spill_kvarn(int bits, const LayerView &L, const Work &W, const __nv_
 }  // namespace
 
 int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &seqs, const void *k,
-                  const void *v, cudaStream_t st) {
+                  const void *v, cudaStream_t st, AppendInfo *info) {
+  AppendInfo local;
+  AppendInfo &I = info ? *info : local;
+  I = AppendInfo{};
   const LayerView L = layer_view(c, layer);
   const __nv_bfloat16 *in[2] = {static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v)};
   const int fam[2] = {c->fam_k, c->fam_v}, bits[2] = {c->bits_k, c->bits_v};
@@ -612,8 +710,18 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
 
   for (size_t base = 0; base < seqs.size(); base += MAXS) {
     const size_t cnt = std::min<size_t>(MAXS, seqs.size() - base);
-    // 1. spill quantization: K and V in one launch when they share a kvarn type
+    // 1. spill quantization: K and V in one launch when they share a kvarn type; that launch
+    //    also writes the new ring rows when every sequence spills and, for each, the rows from
+    //    the first one the spill reads to the last one written span at most the ring
     const bool fused = c->p.type_k == c->p.type_v && fam[0] == FAM_KVARN;
+    bool ring_fused = fused;
+    for (size_t i = 0; i < cnt && ring_fused; ++i) {
+      const AppendSeq &a = seqs[base + i];
+      const int64_t n1 = a.n0 + a.n_new;
+      const int64_t Q0 = quantized_len(c, a.n0), Q1 = quantized_len(c, n1);
+      if (Q1 <= Q0 || n1 - (Q0 / GROUP) * GROUP > c->ring_cap) ring_fused = false;
+    }
+    int spill_ctas = 0;
     for (int which = 0; which < 2; ++which) {
       if (fam[which] == FAM_BF16) continue;
       if (fused && which == 1) continue;
@@ -627,6 +735,8 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
         s.n0 = a.n0;
         s.n1 = a.n0 + a.n_new;
         s.in_off = a.in_off;
+        const int64_t ks = keep_start(c, fam[which], s.n1);
+        s.tw = ring_fused ? (ks > s.n0 ? ks : s.n0) : s.n1;
         const int64_t Q0 = quantized_len(c, s.n0), Q1 = quantized_len(c, s.n1);
         if (Q1 <= Q0) continue;
         int64_t items;
@@ -651,7 +761,14 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
                                         : spill_qb<1>(fam[which], bits[which], L, W, in[which], st));
       if (e != cudaSuccess) return KVQ_E_CUDA;
       note_launches(1);
+      ++I.launches;
+      spill_ctas = fam[which] == FAM_KVARN ? (int)W.total : 0;
     }
+    if (ring_fused) {
+      I.last_ctas = spill_ctas;
+      continue;
+    }
+    I.last_ctas = 0;
     // 2. ring write of the new rows that stay 16-bit (K and V in one launch when their
     //    types keep the same rows)
     const bool same_keep = fam[0] == fam[1];
@@ -681,6 +798,7 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
       k_tail_write<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(L, W, in[0], in[1]);
       if (cudaGetLastError() != cudaSuccess) return KVQ_E_CUDA;
       note_launches(1);
+      ++I.launches;
     }
   }
   return KVQ_OK;

@@ -41,7 +41,17 @@ struct DSeq {
   int32_t cta0;         // first CTA of this sequence
   int32_t part0;        // first partial slot of this sequence
   int64_t n, Q;
+  int64_t dq, dt;       // first quantized token / ring token written by the preceding kernel
 };
+
+// Waits for the kernel this one was launched behind (programmatic stream serialization) and
+// for its memory writes; returns at once when the launch had no such dependency.
+__device__ __forceinline__ void wait_producer() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// First chunk of a range starting at token a whose tokens reach `dirty` (chunks of CH tokens).
+__device__ __forceinline__ int64_t first_dirty_chunk(int64_t a, int64_t dirty) {
+  return dirty <= a ? 0 : (dirty - a) / CH;
+}
 
 struct DArgs {
   int32_t nseq, G, hkv, rotk, rotv, ncta;
@@ -71,17 +81,60 @@ __device__ __forceinline__ float warp_sum(float v) {
 //            a3 = (row g+8, k 16+4tq..);  B 32x8: b0 = (k 4tq.., col g), b1 = (k 16+4tq.., col g);
 //   C 16x8: c0 = (row g, col 2tq), c1 = (g, 2tq+1), c2 = (g+8, 2tq), c3 = (g+8, 2tq+1).
 // Rows 0..7 carry the high int8 limb and rows 8..15 the low limb of a 16-bit fixed-point
-// operand of query head g (Q for Q.K, the softmax weights for P.V); both MMA results of one
-// column combine exactly in int32 as 256*hi + lo.
+// operand of query head g (Q for Q.K, the softmax weights for P.V); the two int32 results of
+// one column combine as 256*hi + lo with one fp32 rounding.
 
-// d = a.b + (bias in every element): the accumulator input is one shared register, so no
-// per-MMA reinitialization is needed
-__device__ __forceinline__ void mma_s8_bias(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, int bias) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%10,%10,%10,%10};\n"
-      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(bias));
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: two lanes per instruction, each lane
+//      rounded once exactly as the scalar operation) ----------------------------------------
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pk2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(f32x2 v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ float acc_part(f32x2 v, int e) {
+  float lo, hi;
+  upk2(v, lo, hi);
+  return e ? hi : lo;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// One block of Q.K or P.V on the tensor cores with its epilogue on packed fp32:
+//   x += f * (256 * hi + lo)
+// for the two columns of this lane (c0/c2 = hi/lo of column 2tq, c1/c3 = hi/lo of column
+// 2tq+1).  The int32 accumulators start at the bits of 1.5 * 2^23, so each result read as
+// a float is 1.5 * 2^23 + value (exact for |value| < 2^22) and one subtraction recovers it.
+__device__ __forceinline__ void mma_s8_fold(f32x2 &x, const uint32_t (&a)[4], uint32_t b0, uint32_t b1, f32x2 f) {
+  const f32x2 bias = 0x4B4000004B400000ull;  // (1.5 * 2^23, 1.5 * 2^23)
+  const f32x2 k256 = 0x4380000043800000ull;  // (256, 256)
+  asm("{\n"
+      " .reg .b32 c0, c1, c2, c3;\n"
+      " .reg .b64 h, l;\n"
+      " mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {c0,c1,c2,c3}, {%1,%2,%3,%4}, {%5,%6}, "
+      "{%7,%7,%7,%7};\n"
+      " mov.b64 h, {c0, c1};\n"
+      " mov.b64 l, {c2, c3};\n"
+      " sub.rn.f32x2 h, h, %8;\n"
+      " sub.rn.f32x2 l, l, %8;\n"
+      " fma.rn.f32x2 h, h, %9, l;\n"
+      " fma.rn.f32x2 %0, %10, h, %0;\n"
+      "}\n"
+      : "+l"(x)
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0x4B400000), "l"(bias), "l"(k256),
+        "l"(f));
 }
 
 // field s (width W) of each byte of `word`, moved to bits [P, P+W) of the same byte
@@ -285,14 +338,12 @@ __device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head
 
 // Per-warp scale tables of one chunk, built with one token per lane.
 struct ChunkTabs {
-  float k[CH][4];   // K: d * t (kvarn) or d, per token and block (0 past the context end)
+  float k[CH / 2][4][2];  // K: d * t (kvarn) or d, per token pair, block, token (0 past the end)
   float v[4][CH];   // V: t * d * QFIX / max over the chunk (per block) -> weights in fixed point
   float km[CH][4];  // qb_1 K: m + d * 2^(b-1)
   float vm[CH][4];  // qb_1 V: m + d * 2^(b-1)
 };
 
-constexpr int kBias = 0x4B400000;       // float bits of 1.5 * 2^23
-constexpr float kBiasF = 12582912.0f;  // an int32 accumulator started at kBias reads as kBiasF + sum
 
 // Query fragments of one page: the query of head g times the page's K channel scales c
 // (kvarn), in 16-bit fixed point relative to the head's max, split into int8 limbs (hi in
@@ -364,11 +415,18 @@ __device__ __forceinline__ void make_qfrag(QFrag &f, const float (*qrot)[D], con
 // groups past the end), so that their copies overlap the query prologue.
 template <int FAM, int BITS>
 __device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq, int head, int64_t a, int c0, int c1,
-                                                    uint8_t *stages, int lane, PageCursor &pc) {
+                                                    int64_t cdirty, bool &waited, uint8_t *stages, int lane,
+                                                    PageCursor &pc) {
   using S = Stage<FAM, BITS>;
 #pragma unroll
   for (int j = 0; j < S::NST - 1; ++j) {
-    if (c0 + j < c1) copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)(c0 + j) * CH, stages + j * S::BYTES, lane, pc);
+    if (c0 + j < c1) {
+      if (c0 + j >= cdirty && !waited) {
+        wait_producer();
+        waited = true;
+      }
+      copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)(c0 + j) * CH, stages + j * S::BYTES, lane, pc);
+    }
     cp_async_commit();
   }
 }
@@ -378,8 +436,9 @@ __device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq,
 // stored basis) of its heads to shared memory.
 template <int FAM, int BITS>
 __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head, int64_t a, int64_t b, int c0,
-                                           int c1, int G, const float (*qrot)[D], uint8_t *stages, ChunkTabs &T,
-                                           float *mw, float *lw, float *accw, PageCursor &pc) {
+                                           int c1, int64_t cdirty, bool waited, int G, const float (*qrot)[D],
+                                           uint8_t *stages, ChunkTabs &T, float *mw, float *lw, float *accw,
+                                           PageCursor &pc) {
   using S = Stage<FAM, BITS>;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -388,9 +447,9 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
   constexpr float HALF_RANGE = (float)(1 << (BITS - 1));
   constexpr float SCL = CSC / QFIX;
 
-  float acc[32];  // index blk*8 + u*2 + e <-> channel 32 blk + 8 tq + 4 e + u
+  f32x2 acc[16];  // index blk*4 + u <-> channels (32 blk + 8 tq + u, 32 blk + 8 tq + 4 + u)
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+  for (int i = 0; i < 16; ++i) acc[i] = 0ull;
   float aoff[4] = {0.f, 0.f, 0.f, 0.f};
   float m_run = -INFINITY, l_run = 0.f;
   QFrag qf;
@@ -402,7 +461,13 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     {  // keep NST - 1 chunks in flight: issue chunk c + NST - 1 into the stage read last round
       const int cn = c + S::NST - 1;
       const int sn = si == 0 ? S::NST - 1 : si - 1;
-      if (cn < c1) copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)cn * CH, stages + sn * S::BYTES, lane, pc);
+      if (cn < c1) {
+        if (cn >= cdirty && !waited) {
+          wait_producer();
+          waited = true;
+        }
+        copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)cn * CH, stages + sn * S::BYTES, lane, pc);
+      }
       cp_async_commit();
       cp_async_wait<S::NST - 1>();  // chunk c has landed (for this lane's copies)
       __syncwarp();                 // ... and for every lane's
@@ -435,7 +500,8 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       // select (not multiply) so that NaN bit patterns in stale rows cannot leak
       const float dkt[4] = {vl ? dk01.x * tkl : 0.f, vl ? dk01.y * tkl : 0.f, vl ? dk23.x * tkl : 0.f,
                             vl ? dk23.y * tkl : 0.f};
-      *reinterpret_cast<float4 *>(&T.k[lane][0]) = make_float4(dkt[0], dkt[1], dkt[2], dkt[3]);
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) T.k[lane >> 1][blk][lane & 1] = dkt[blk];
       float tdv[4] = {vl ? dv01.x * tvl : 0.f, vl ? dv01.y * tvl : 0.f, vl ? dv23.x * tvl : 0.f,
                       vl ? dv23.y * tvl : 0.f};
       float inv[4];
@@ -474,22 +540,17 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       KTok<FAM, BITS> kt;
       kt.load(st + S::KC + (16 * (r >> 1) + 4 * (g >> 1) + 2 * (r & 1) + (g & 1)) * 16 * BITS, tq);
       const int t0 = 16 * (r >> 1) + 4 * tq + 2 * (r & 1);
-      const float4 dA = *reinterpret_cast<const float4 *>(&T.k[t0][0]);
-      const float4 dB = *reinterpret_cast<const float4 *>(&T.k[t0 + 1][0]);
-      const float d0[4] = {dA.x, dA.y, dA.z, dA.w}, d1[4] = {dB.x, dB.y, dB.z, dB.w};
-      float x0 = 0.f, x1 = 0.f;
+      // (d of token t0, d of token t0 + 1) per block, as packed pairs
+      const f32x2 *dp = reinterpret_cast<const f32x2 *>(&T.k[t0 >> 1][0][0]);
+      f32x2 x = 0ull;
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
         uint32_t b0, b1;
         kt.frag(blk, tq, b0, b1);
-        int c[4];
-        mma_s8_bias(c, qf.qa[blk], b0, b1, kBias);
-        const float h0 = __int_as_float(c[0]) - kBiasF, h1 = __int_as_float(c[1]) - kBiasF;
-        const float l0 = __int_as_float(c[2]) - kBiasF, l1 = __int_as_float(c[3]) - kBiasF;
-        x0 = fmaf(d0[blk], fmaf(256.f, h0, l0), x0);
-        x1 = fmaf(d1[blk], fmaf(256.f, h1, l1), x1);
+        mma_s8_fold(x, qf.qa[blk], b0, b1, dp[blk]);
       }
-      float s0 = x0 * sigp, s1 = x1 * sigp;
+      float s0, s1;
+      upk2(mul2(x, pk2(sigp, sigp)), s0, s1);
       if (FAM == FAM_ASYM) {
         const float4 mA = *reinterpret_cast<const float4 *>(&T.km[t0][0]);
         const float4 mB = *reinterpret_cast<const float4 *>(&T.km[t0 + 1][0]);
@@ -516,7 +577,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     }
     if (__any_sync(FULL, alpha != 1.f)) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] *= alpha;
+      for (int i = 0; i < 16; ++i) acc[i] = mul2(acc[i], pk2(alpha, alpha));
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) aoff[blk] *= alpha;
     }
@@ -541,7 +602,12 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       const float tvk[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
       uint32_t wb[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) wb[k] = __float_as_uint(fmaf(p[k], tvk[k], MAGIC));
+      for (int k = 0; k < 8; k += 2) {
+        float w0, w1;
+        upk2(fma2(pk2(p[k], p[k + 1]), pk2(tvk[k], tvk[k + 1]), pk2(MAGIC, MAGIC)), w0, w1);
+        wb[k] = __float_as_uint(w0);
+        wb[k + 1] = __float_as_uint(w1);
+      }
       uint32_t wa[4];
       {
         const uint32_t x = __byte_perm(wb[0], wb[1], 0x5140), y = __byte_perm(wb[2], wb[3], 0x5140);
@@ -553,33 +619,26 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
         wa[2] = __byte_perm(x, y, 0x7632);
         wa[3] = __byte_perm(x, y, 0x5410) ^ 0x80808080u;
       }
-      // per-channel factor: the block's fixed-point scale, times the page's V channel scale c
-      float f[8];
+      // per-channel factor of the lane's two columns (channels 8 tq + u and 8 tq + 4 + u of
+      // the block): the block's fixed-point scale, times the page's V channel scale c
+      f32x2 f[4];
       if (FAM == FAM_KVARN) {
         const uint4 c8 = *reinterpret_cast<const uint4 *>(st + S::VCS + 2 * (32 * blk + 8 * tq));
-        const __half2 *c2 = reinterpret_cast<const __half2 *>(&c8);
+        const __half *ch = reinterpret_cast<const __half *>(&c8);
 #pragma unroll
-        for (int q2 = 0; q2 < 4; ++q2) {
-          const float2 cf = __half22float2(c2[q2]);
-          f[2 * q2] = scl[blk] * cf.x;
-          f[2 * q2 + 1] = scl[blk] * cf.y;
-        }
+        for (int u = 0; u < 4; ++u)
+          f[u] = mul2(pk2(scl[blk], scl[blk]), pk2(__half2float(ch[u]), __half2float(ch[u + 4])));
       } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = scl[blk];
+        for (int u = 0; u < 4; ++u) f[u] = pk2(scl[blk], scl[blk]);
       }
       VQuad<FAM, BITS> v0, v1;
       v0.load(st + S::VC + tq * S::QS, blk, g);
       v1.load(st + S::VC + (4 + tq) * S::QS, blk, g);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        int c[4];
-        mma_s8_bias(c, wa, v0.frag(u, g), v1.frag(u, g), kBias);
-        const float h0 = __int_as_float(c[0]) - kBiasF, h1 = __int_as_float(c[1]) - kBiasF;
-        const float l0 = __int_as_float(c[2]) - kBiasF, l1 = __int_as_float(c[3]) - kBiasF;
         // column 2tq <-> channel 32 blk + 8 tq + u, column 2tq+1 <-> + 4
-        acc[blk * 8 + u * 2 + 0] = fmaf(f[u], fmaf(256.f, h0, l0), acc[blk * 8 + u * 2 + 0]);
-        acc[blk * 8 + u * 2 + 1] = fmaf(f[4 + u], fmaf(256.f, h1, l1), acc[blk * 8 + u * 2 + 1]);
+        mma_s8_fold(acc[blk * 4 + u], wa, v0.frag(u, g), v1.frag(u, g), f[u]);
       }
     }
 
@@ -605,7 +664,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int e = 0; e < 2; ++e)
-          accw[g * D + 32 * blk + 8 * tq + 4 * e + u] = acc[blk * 8 + u * 2 + e] + aoff[blk];
+          accw[g * D + 32 * blk + 8 * tq + 4 * e + u] = acc_part(acc[blk * 4 + u], e) + aoff[blk];
     if (tq == 0) {
       mw[g] = m_run;
       lw[g] = l_run;
@@ -616,8 +675,8 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
 // Exact BF16 rows (the tail, or a whole BF16 cache) on CUDA cores: Q.K with one token per
 // lane, P.V with four channels per lane.  Tokens [c0*32 + a, ...) of this warp.
 __device__ __forceinline__ void warp_bf16(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
-                                          int64_t c1, int G, const float (*qraw)[D], float (*pst)[MAX_G],
-                                          float *mw, float *lw, float *accw) {
+                                          int64_t c1, int64_t cdirty, int G, const float (*qraw)[D],
+                                          float (*pst)[MAX_G], float *mw, float *lw, float *accw) {
   const int lane = threadIdx.x & 31;
   float m[MAX_G], l[MAX_G], acc[MAX_G][4];
 #pragma unroll
@@ -631,6 +690,7 @@ __device__ __forceinline__ void warp_bf16(const LayerView &L, int seq, int head,
   const __nv_bfloat16 *vbase = ring_row(L, seq, head, 1, 0);
 #pragma unroll 1
   for (int64_t ci = c0; ci < c1; ++ci) {
+    if (ci == (cdirty > c0 ? cdirty : c0) && cdirty < c1) wait_producer();
     const int64_t i0 = a + ci * CH;
     const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
     const bool valid = lane < nvalid;
@@ -818,13 +878,17 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
     b = min(a + (int64_t)s.cps_t * CH, s.n);
   }
   nch = b > a ? (b - a + CH - 1) / CH : 0;
-  // a contiguous chunk range per warp
-  const int64_t per = (nch + NW - 1) / NW;
-  const int64_t c0 = min((int64_t)warp * per, nch), c1 = min(c0 + per, nch);
+  // a contiguous chunk range per warp, sizes differing by at most one
+  const int64_t c0 = nch * warp / NW, c1 = nch * (warp + 1) / NW;
 
+  // chunks at or past cdirty hold tokens the preceding (overlapped) append kernel writes
+  const int64_t cdirty = first_dirty_chunk(a, (tail || FAM == FAM_BF16) ? s.dt : s.dq);
+  bool waited = false;
   PageCursor pc;
   if constexpr (FAM != FAM_BF16) {
-    if (!tail) warp_quant_prefetch<FAM, BITS>(L, s.seq, head, a, (int)c0, (int)c1, warp_mem + (size_t)warp * WA, lane, pc);
+    if (!tail)
+      warp_quant_prefetch<FAM, BITS>(L, s.seq, head, a, (int)c0, (int)c1, cdirty, waited, warp_mem + (size_t)warp * WA,
+                                     lane, pc);
   }
   // query rows of this KV head, pre-scaled by softmax_scale * log2(e); heads >= G are 0
   for (int idx = tid; idx < MAX_G * D; idx += DT) {
@@ -857,17 +921,17 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
   static_assert(WA >= MAX_G * D * 4 + CH * MAX_G * 4, "warp area holds accumulator and weights");
   if constexpr (FAM != FAM_BF16) {
     if (!tail) {
-      warp_quant<FAM, BITS>(L, s.seq, head, a, b, (int)c0, (int)c1, G, F.qrot, warp_mem + (size_t)warp * WA,
-                            F.tabs[warp], F.mw[warp], F.lw[warp], accw, pc);
+      warp_quant<FAM, BITS>(L, s.seq, head, a, b, (int)c0, (int)c1, cdirty, waited, G, F.qrot,
+                            warp_mem + (size_t)warp * WA, F.tabs[warp], F.mw[warp], F.lw[warp], accw, pc);
     } else {
       for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
       __syncwarp();
-      warp_bf16(L, s.seq, head, a, b, c0, c1, G, F.qraw, pst, F.mw[warp], F.lw[warp], accw);
+      warp_bf16(L, s.seq, head, a, b, c0, c1, cdirty, G, F.qraw, pst, F.mw[warp], F.lw[warp], accw);
     }
   } else {
     for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
     __syncwarp();
-    warp_bf16(L, s.seq, head, a, b, c0, c1, G, F.qraw, pst, F.mw[warp], F.lw[warp], accw);
+    warp_bf16(L, s.seq, head, a, b, c0, c1, cdirty, G, F.qraw, pst, F.mw[warp], F.lw[warp], accw);
   }
   __syncthreads();
 
@@ -1002,7 +1066,7 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
 }
 
 template <int FAM, int BITS>
-cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st) {
+cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
   constexpr size_t smem = smem_bytes<FAM, BITS>();
   static_assert(smem <= 232448, "shared memory per CTA");
   static_assert((nwarps(FAM, BITS) * warp_area<FAM, BITS>()) / (PSTRIDE * 4) >= MAX_G, "merge stage holds a split");
@@ -1013,13 +1077,22 @@ cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_decode<FAM, BITS><<<A.ncta, 32 * nwarps(FAM, BITS), smem, st>>>(L, A);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)A.ncta);
+  cfg.blockDim = dim3(32 * nwarps(FAM, BITS));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  la[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = la;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_decode<FAM, BITS>, L, A);
 }
 
-cudaError_t dispatch(int fam, int bits, const LayerView &L, const DArgs &A, cudaStream_t st) {
+cudaError_t dispatch(int fam, int bits, const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
 #define KVQ_D(F, B) \
-  if (fam == F && bits == B) return run<F, B>(L, A, st);
+  if (fam == F && bits == B) return run<F, B>(L, A, st, pdl);
   KVQ_D(FAM_BF16, 16)
   KVQ_D(FAM_SYM, 2) KVQ_D(FAM_SYM, 3) KVQ_D(FAM_SYM, 4) KVQ_D(FAM_SYM, 5) KVQ_D(FAM_SYM, 6) KVQ_D(FAM_SYM, 8)
   KVQ_D(FAM_ASYM, 2) KVQ_D(FAM_ASYM, 3) KVQ_D(FAM_ASYM, 4) KVQ_D(FAM_ASYM, 5) KVQ_D(FAM_ASYM, 6)
@@ -1037,14 +1110,18 @@ size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads) {
 }
 
 int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &seqs, int n_q_heads,
-                  const float *q, float scale, float *out, void *ws, size_t ws_bytes, cudaStream_t st) {
+                  const float *q, float scale, float *out, void *ws, size_t ws_bytes, cudaStream_t st,
+                  int budget_sms, bool pdl) {
+  const int sms = budget_sms > 0 && budget_sms < c->num_sms ? budget_sms : c->num_sms;
   if (c->p.type_k != c->p.type_v) return KVQ_E_UNSUPPORTED;
   (void)ws_bytes;
   const LayerView L = layer_view(c, layer);
   const int hkv = c->p.n_kv_heads, G = n_q_heads / hkv;
-  // bytes per token of a (K+V) head pair; BF16 rows weigh double (CUDA-core path)
+  // relative cost of one token of a (K+V) head pair: quantized tokens by their bytes; BF16
+  // tail tokens on the CUDA-core path take about 5.5 times as long as a quantized token
+  // (measured: ~20 vs ~108 tokens per microsecond and SM)
   const double tbq = (double)token_bytes(c->fam_k, c->bits_k) + token_bytes(c->fam_v, c->bits_v);
-  const double tbt = 2.0 * 4.0 * D;
+  const double tbt = 5.5 * tbq;
   for (size_t base = 0; base < seqs.size(); base += MAXS) {
     const size_t cnt = std::min<size_t>(MAXS, seqs.size() - base);
     DArgs A{};
@@ -1058,40 +1135,31 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
     A.out = out;
     A.ws = static_cast<float *>(ws);
     A.tickets = reinterpret_cast<uint32_t *>(c->base + c->off_tickets);
-    // split plan: about one CTA per SM in total, shared out by weighted bytes; every
-    // (sequence, part) with tokens gets at least one split per KV head
-    double wsum = 0.0;
-    for (size_t i = 0; i < cnt; ++i) {
-      const DecodeSeq &d = seqs[base + i];
-      wsum += (double)d.Q * tbq + (double)(d.n - d.Q) * tbt;
-    }
-    const double per_head = (double)c->num_sms / hkv;
+    // split plan (min-max greedy): every (sequence, part) with tokens starts with one split
+    // per KV head; then, while a whole column of hkv CTAs still fits in one wave, the part
+    // whose splits carry the most work gets one more split
     std::vector<int> nq(cnt), nt(cnt);
-    std::vector<double> rq(cnt), rt(cnt);
     int used = 0;
     for (size_t i = 0; i < cnt; ++i) {
       const DecodeSeq &d = seqs[base + i];
-      const int64_t nchq = (d.Q + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
-      const double sq = wsum > 0 ? per_head * d.Q * tbq / wsum : 0.0;
-      const double st_ = wsum > 0 ? per_head * (d.n - d.Q) * tbt / wsum : 0.0;
-      nq[i] = nchq ? (int)std::min<int64_t>(std::max(1, std::min((int)sq, MAXSQ)), nchq) : 0;
-      nt[i] = ncht ? (int)std::min<int64_t>(std::max(1, std::min((int)st_, MAXST)), ncht) : 0;
-      rq[i] = nchq ? sq - nq[i] : -1.0;
-      rt[i] = ncht ? st_ - nt[i] : -1.0;
+      nq[i] = d.Q > 0 ? 1 : 0;
+      nt[i] = d.n > d.Q ? 1 : 0;
       used += hkv * (nq[i] + nt[i]);
     }
-    // hand the CTAs left by rounding down to the largest remainders
-    while (used + hkv <= c->num_sms) {
+    while (used + hkv <= sms) {
       int best = -1;
       bool best_t = false;
-      double br = 0.0;
+      double most = 0.0;
       for (size_t i = 0; i < cnt; ++i) {
         const DecodeSeq &d = seqs[base + i];
-        if (rq[i] > br && nq[i] < MAXSQ && nq[i] < (d.Q + CH - 1) / CH) { br = rq[i]; best = (int)i; best_t = false; }
-        if (rt[i] > br && nt[i] < MAXST && nt[i] < (d.n - d.Q + CH - 1) / CH) { br = rt[i]; best = (int)i; best_t = true; }
+        const int64_t nchq = (d.Q + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
+        const double wq = nq[i] ? (double)d.Q * tbq / nq[i] : 0.0;
+        const double wt = nt[i] ? (double)(d.n - d.Q) * tbt / nt[i] : 0.0;
+        if (wq > most && nq[i] < MAXSQ && nq[i] < nchq) { most = wq; best = (int)i; best_t = false; }
+        if (wt > most && nt[i] < MAXST && nt[i] < ncht) { most = wt; best = (int)i; best_t = true; }
       }
       if (best < 0) break;
-      if (best_t) { ++nt[best]; rt[best] -= 1.0; } else { ++nq[best]; rq[best] -= 1.0; }
+      if (best_t) ++nt[best]; else ++nq[best];
       used += hkv;
     }
     int cta = 0, part = 0;
@@ -1102,6 +1170,8 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
       s.row = d.row;
       s.n = d.n;
       s.Q = d.Q;
+      s.dq = d.dq;
+      s.dt = d.dt;
       const int64_t nchq = (d.Q + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
       s.cps_q = nq[i] ? (int)((nchq + nq[i] - 1) / nq[i]) : 1;
       s.nsq = nq[i] ? (int)((nchq + s.cps_q - 1) / s.cps_q) : 0;
@@ -1115,7 +1185,9 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
     }
     A.ncta = cta;
     // q / out rows are indexed by DecodeSeq::row; the workspace slots restart per launch
-    if (dispatch(c->fam_k, c->bits_k, L, A, st) != cudaSuccess) return KVQ_E_CUDA;
+    // overlap only a decode of one launch: a second launch would follow the first, not the producer
+    if (dispatch(c->fam_k, c->bits_k, L, A, st, pdl && seqs.size() <= (size_t)MAXS) != cudaSuccess)
+      return KVQ_E_CUDA;
     note_launches(1);
   }
   return KVQ_OK;

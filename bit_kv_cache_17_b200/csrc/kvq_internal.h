@@ -55,18 +55,36 @@ struct AppendSeq {
   int64_t in_off;  // first input row of this sequence
 };
 
-// Launchers; return KVQ_OK or a KVQ_E_* code.
-int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &seqs,
-                  const void *k, const void *v, cudaStream_t st);
+// What an append left in flight, for a decode launched right behind it.
+struct AppendInfo {
+  int launches = 0;      // kernels launched by the append
+  int last_ctas = 0;     // CTAs of its last kernel when that kernel is the fused spill + ring
+                         // write of a few groups (they hold their SMs while a decode overlaps)
+};
 
+// Launchers; return KVQ_OK or a KVQ_E_* code.  Every append kernel signals its dependents
+// (griddepcontrol.launch_dependents) as it starts, so that a decode launched with
+// programmatic stream serialization behind it may begin early.
+int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &seqs,
+                  const void *k, const void *v, cudaStream_t st, AppendInfo *info = nullptr);
+
+constexpr int64_t kNeverDirty = INT64_MAX;
 struct DecodeSeq {
   int32_t seq;      // sequence slot in the cache
   int32_t row;      // row of q/out for this sequence
   int64_t n;        // tokens
   int64_t Q;        // quantized tokens
+  // Tokens written by the kernel(s) right before this decode in the stream (an overlapped
+  // append): quantized tokens >= dq and BF16 ring rows of tokens >= dt.  A warp waits for
+  // those kernels (griddepcontrol.wait) before it reads such a token.
+  int64_t dq = kNeverDirty, dt = kNeverDirty;
 };
+// budget_sms: SMs the split plan may fill (0 = all); pdl: launch with programmatic stream
+// serialization (the previous kernel in the stream must be an append kernel of this library
+// and every token it wrote must be covered by the sequences' dq / dt).
 int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &seqs, int n_q_heads,
-                  const float *q, float scale, float *out, void *ws, size_t ws_bytes, cudaStream_t st);
+                  const float *q, float scale, float *out, void *ws, size_t ws_bytes, cudaStream_t st,
+                  int budget_sms = 0, bool pdl = false);
 size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads);
 
 int launch_dequant(const kvq_cache *c, int layer, int seq, int which, int64_t t0, int64_t t1,

@@ -140,6 +140,25 @@ int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *
                     int32_t n_q_heads, const float *q, float softmax_scale, float *out,
                     void *workspace, size_t ws_bytes, kvq_stream_t stream);
 
+/* One decode step of a layer: kvq_append (n_new[i] tokens to seq_ids[i]) followed by
+ * kvq_decode_attn of the same sequences (q / out row i belongs to seq_ids[i]), with the
+ * same arguments, layouts and results as the two calls.  The pages ("KV Cache Precision
+ * Tail": the newest tokens are written 16-bit, the oldest tail token spills into its
+ * quantized group; the long-context decode discussion: decode attention reads the whole
+ * cache) make these the two halves of every generated token.
+ * The decode is launched with programmatic stream serialization behind the append's last
+ * kernel: its warps start on pages the append does not touch while the append runs, and
+ * wait for it (griddepcontrol.wait) only before the pages and ring rows it rewrites.  When
+ * that kernel is a small spill (a one-token step), the decode's split plan leaves the
+ * spill's SMs out.  Requirements beyond the two calls': q must be complete before this call
+ * is issued (it is read while the append runs), and nothing else may be enqueued on `stream`
+ * in between (there is nothing in between: this is one call).  Errors: those of the two
+ * calls, all checked before anything is launched. */
+int kvq_append_decode(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,
+                      const int32_t *n_new, const void *k_bf16, const void *v_bf16, int32_t n_q_heads,
+                      const float *q, float softmax_scale, float *out, void *workspace, size_t ws_bytes,
+                      kvq_stream_t stream);
+
 /* Dequantizes tokens [t0, t1) of K (which = 0) or V (which = 1) of one sequence into
  * out: device fp32 [t1 - t0, n_kv_heads, 128].  basis 0 = original basis (kvarn values
  * are rotated back with the same fp32 butterfly), basis 1 = the stored rotated basis.
