@@ -261,7 +261,8 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 // Shared-memory image of one 32-token chunk of a quantized page (both K and V), filled by
 // cp.async: codes of K, codes of V one quad per row with a 32-byte pad (so that the lanes
-// of one P.V fragment load hit distinct banks), then the fp16 scales.
+// of one P.V fragment load hit distinct banks), then the fp16 scales (d of K then V; m of K
+// then V for qb_1; t of K then V for kvarn).
 template <int FAM, int BITS>
 struct Stage {
   static constexpr int QS = 64 * BITS + 32;  // padded quad stride
@@ -273,10 +274,17 @@ struct Stage {
   static constexpr int VM = KM + (FAM == FAM_ASYM ? 256 : 0);
   static constexpr int KT = VM + (FAM == FAM_ASYM ? 256 : 0);
   static constexpr int VT = KT + (FAM == FAM_KVARN ? 64 : 0);
-  static constexpr int KCS = VT + (FAM == FAM_KVARN ? 64 : 0);
-  static constexpr int VCS = KCS + (FAM == FAM_KVARN ? 256 : 0);
-  static constexpr int BYTES = VCS + (FAM == FAM_KVARN ? 256 : 0);
+  static constexpr int BYTES = VT + (FAM == FAM_KVARN ? 64 : 0);
   static constexpr int NST = BITS <= 3 ? 3 : 2;  // stages per warp
+};
+
+// Per-warp data of whole pages (kvarn): the channel scales c of K and V of the pages being
+// copied (double-buffered by page parity: copies run at most NST - 1 chunks ahead of the
+// compute, so they never reach a third page), and the V channel scales of the page being
+// computed as the fp32 pairs each lane's P.V columns need.
+struct PageArea {
+  __half c[2][2][D];  // [page & 1][K, V][channel]
+  float2 fv[4][16];   // [tq][blk * 4 + u] = (c_V[32 blk + 8 tq + u], c_V[32 blk + 8 tq + 4 + u])
 };
 
 // Source cursor of a warp's copies: the K and V sub-pages of the page being copied, looked up
@@ -284,55 +292,52 @@ struct Stage {
 struct PageCursor {
   int64_t page = -1;
   const uint8_t *sk = nullptr, *sv = nullptr;
-  __device__ __forceinline__ void seek(const LayerView &L, int seq, int head, int64_t p) {
-    if (p != page) {
-      page = p;
-      sk = subpage_ptr(L, seq, p, head, 0);
-      sv = sk + L.sub_k;
-    }
+  __device__ __forceinline__ bool seek(const LayerView &L, int seq, int head, int64_t p) {
+    if (p == page) return false;
+    page = p;
+    sk = subpage_ptr(L, seq, p, head, 0);
+    sv = sk + L.sub_k;
+    return true;
   }
 };
 
-// Copies chunk [i0, i0+32) (K and V codes, fp16 scales, and for kvarn the page's channel
-// scales) into the stage `st`, 16 bytes per lane and instruction, as one commit group.
+// Copies chunk [i0, i0+32) (K and V codes and fp16 scales; for kvarn, on the first chunk of a
+// page, the page's channel scales) into the stage `st`, 16 bytes per lane and instruction, as
+// one commit group.
 template <int FAM, int BITS>
 __device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head, int64_t i0, uint8_t *st, int lane,
-                                           PageCursor &pc) {
+                                           PageCursor &pc, PageArea *pa) {
   using S = Stage<FAM, BITS>;
   const SubLayout lay = sub_layout(FAM, BITS);
-  pc.seek(L, seq, head, i0 / GROUP);
+  const int64_t page = i0 / GROUP;
+  if (pc.seek(L, seq, head, page) && FAM == FAM_KVARN)
+    cp_async16(&pa->c[page & 1][lane >> 4][8 * (lane & 15)], (lane < 16 ? pc.sk : pc.sv) + lay.c + 16 * (lane & 15));
   const int tip0 = (int)(i0 % GROUP);
-  const uint8_t *sk = pc.sk;
-  const uint8_t *sv = pc.sv;
   constexpr int KP = 32 * BITS;  // 16-byte pieces of K codes (and of V codes)
   constexpr int QP = 4 * BITS;   // pieces per V quad
-  const uint8_t *kc = sk + tip0 * 16 * BITS;
-  const uint8_t *vc = sv + (tip0 / 4) * 64 * BITS;
+  // K and V codes of the chunk are contiguous (tip0 is a multiple of 4: V quads are whole)
+  const uint8_t *kc = pc.sk + tip0 * 16 * BITS + 16 * lane;
+  const uint8_t *vc = pc.sv + tip0 * 16 * BITS + 16 * lane;
 #pragma unroll
-  for (int p = lane; p < KP; p += 32) cp_async16(st + S::KC + 16 * p, kc + 16 * p);
+  for (int j = 0; j < KP / 32; ++j) cp_async16(st + S::KC + 16 * lane + 512 * j, kc + 512 * j);
+  if constexpr (32 % QP == 0) {
+    uint8_t *vd = st + S::VC + (lane / QP) * S::QS + 16 * (lane % QP);
 #pragma unroll
-  for (int p = lane; p < KP; p += 32) {
-    const int q = p / QP, o = p % QP;
-    cp_async16(st + S::VC + q * S::QS + 16 * o, vc + q * 64 * BITS + 16 * o);
+    for (int j = 0; j < KP / 32; ++j) cp_async16(vd + j * (32 / QP) * S::QS, vc + 512 * j);
+  } else {
+#pragma unroll
+    for (int j = 0; j < KP / 32; ++j) {
+      const int p = lane + 32 * j, q = p / QP, o = p % QP;
+      cp_async16(st + S::VC + q * S::QS + 16 * o, vc + 512 * j);
+    }
   }
-  // fp16 scales: 16 pieces of d for K and V, + m (qb_1), + t, c (kvarn)
-  if (lane < 16) {
-    cp_async16(st + S::KD + 16 * lane, sk + lay.d + tip0 * 8 + 16 * lane);
-    cp_async16(st + S::VD + 16 * lane, sv + lay.d + tip0 * 8 + 16 * lane);
-    if constexpr (FAM == FAM_ASYM) {
-      cp_async16(st + S::KM + 16 * lane, sk + lay.m + tip0 * 8 + 16 * lane);
-      cp_async16(st + S::VM + 16 * lane, sv + lay.m + tip0 * 8 + 16 * lane);
-    }
-    if constexpr (FAM == FAM_KVARN) {
-      cp_async16(st + S::KCS + 16 * lane, sk + lay.c + 16 * lane);
-      cp_async16(st + S::VCS + 16 * lane, sv + lay.c + 16 * lane);
-    }
-  } else if (FAM == FAM_KVARN && lane < 24) {
-    const int l = lane - 16;  // 4 pieces each of t for K and V
-    if (l < 4)
-      cp_async16(st + S::KT + 16 * l, sk + lay.t + tip0 * 2 + 16 * l);
-    else
-      cp_async16(st + S::VT + 16 * (l - 4), sv + lay.t + tip0 * 2 + 16 * (l - 4));
+  // fp16 scales: d (and m for qb_1) of K in lanes 0..15, of V in lanes 16..31; t of K in lanes
+  // 0..3, of V in lanes 4..7 (kvarn)
+  const uint8_t *sb = (lane < 16 ? pc.sk : pc.sv) + tip0 * 8 + 16 * (lane & 15);
+  cp_async16(st + S::KD + 16 * lane, sb + lay.d);
+  if constexpr (FAM == FAM_ASYM) cp_async16(st + S::KM + 16 * lane, sb + lay.m);
+  if constexpr (FAM == FAM_KVARN) {
+    if (lane < 8) cp_async16(st + S::KT + 16 * lane, (lane < 4 ? pc.sk : pc.sv) + lay.t + tip0 * 2 + 16 * (lane & 3));
   }
 }
 
@@ -416,7 +421,7 @@ __device__ __forceinline__ void make_qfrag(QFrag &f, const float (*qrot)[D], con
 template <int FAM, int BITS>
 __device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq, int head, int64_t a, int c0, int c1,
                                                     int64_t cdirty, bool &waited, uint8_t *stages, int lane,
-                                                    PageCursor &pc) {
+                                                    PageCursor &pc, PageArea *pa) {
   using S = Stage<FAM, BITS>;
 #pragma unroll
   for (int j = 0; j < S::NST - 1; ++j) {
@@ -425,7 +430,7 @@ __device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq,
         wait_producer();
         waited = true;
       }
-      copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)(c0 + j) * CH, stages + j * S::BYTES, lane, pc);
+      copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)(c0 + j) * CH, stages + j * S::BYTES, lane, pc, pa);
     }
     cp_async_commit();
   }
@@ -438,7 +443,7 @@ template <int FAM, int BITS>
 __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head, int64_t a, int64_t b, int c0,
                                            int c1, int64_t cdirty, bool waited, int G, const float (*qrot)[D],
                                            uint8_t *stages, ChunkTabs &T, float *mw, float *lw, float *accw,
-                                           PageCursor &pc) {
+                                           PageCursor &pc, PageArea *pa) {
   using S = Stage<FAM, BITS>;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -466,7 +471,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
           wait_producer();
           waited = true;
         }
-        copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)cn * CH, stages + sn * S::BYTES, lane, pc);
+        copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)cn * CH, stages + sn * S::BYTES, lane, pc, pa);
       }
       cp_async_commit();
       cp_async_wait<S::NST - 1>();  // chunk c has landed (for this lane's copies)
@@ -477,7 +482,19 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       const int page = (int)(i0 / GROUP);
       const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
       if (page != cur_page && (FAM == FAM_KVARN || cur_page < 0)) {
-        make_qfrag<FAM, BITS>(qf, qrot, reinterpret_cast<const __half *>(st + S::KCS), g, tq, hv);
+        const __half *ck = FAM == FAM_KVARN ? pa->c[page & 1][0] : nullptr;
+        make_qfrag<FAM, BITS>(qf, qrot, ck, g, tq, hv);
+        if constexpr (FAM == FAM_KVARN) {
+          // lane l builds pairs 2 (l >> 2) and 2 (l >> 2) + 1 of column set tq' = l & 3
+          const __half *cv = pa->c[page & 1][1];
+          const int tl = lane & 3;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int idx = 2 * (lane >> 2) + e, blk = idx >> 2, u = idx & 3;
+            pa->fv[tl][idx] = make_float2(__half2float(cv[32 * blk + 8 * tl + u]), __half2float(cv[32 * blk + 8 * tl + 4 + u]));
+          }
+          __syncwarp();
+        }
         cur_page = page;
       }
       const float sigp = qf.sigp;
@@ -567,12 +584,14 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     for (int k = 1; k < 8; ++k) cmax = fmaxf(cmax, sc[k]);
     cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 1));
     cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 2));
+    // every chunk holds a valid token, so mn is finite and exp2(-inf) = 0 covers both the
+    // first chunk (m_run = -inf) and the masked tokens
     const float mn = fmaxf(m_run, cmax);
-    const float alpha = m_run == -INFINITY ? 0.f : exp2_fast(m_run - mn);
+    const float alpha = exp2_fast(m_run - mn);
     float p[8], psum = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      p[k] = sc[k] == -INFINITY ? 0.f : exp2_fast(sc[k] - mn);
+      p[k] = exp2_fast(sc[k] - mn);
       psum += p[k];
     }
     if (__any_sync(FULL, alpha != 1.f)) {
@@ -623,11 +642,9 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       // the block): the block's fixed-point scale, times the page's V channel scale c
       f32x2 f[4];
       if (FAM == FAM_KVARN) {
-        const uint4 c8 = *reinterpret_cast<const uint4 *>(st + S::VCS + 2 * (32 * blk + 8 * tq));
-        const __half *ch = reinterpret_cast<const __half *>(&c8);
+        const f32x2 *cp = reinterpret_cast<const f32x2 *>(&pa->fv[tq][4 * blk]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          f[u] = mul2(pk2(scl[blk], scl[blk]), pk2(__half2float(ch[u]), __half2float(ch[u + 4])));
+        for (int u = 0; u < 4; ++u) f[u] = mul2(pk2(scl[blk], scl[blk]), cp[u]);
       } else {
 #pragma unroll
         for (int u = 0; u < 4; ++u) f[u] = pk2(scl[blk], scl[blk]);
@@ -672,115 +689,173 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
   }
 }
 
-// Exact BF16 rows (the tail, or a whole BF16 cache) on CUDA cores: Q.K with one token per
-// lane, P.V with four channels per lane.  Tokens [c0*32 + a, ...) of this warp.
-__device__ __forceinline__ void warp_bf16(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
-                                          int64_t c1, int64_t cdirty, int G, const float (*qraw)[D],
-                                          float (*pst)[MAX_G], float *mw, float *lw, float *accw) {
-  const int lane = threadIdx.x & 31;
-  float m[MAX_G], l[MAX_G], acc[MAX_G][4];
-#pragma unroll
-  for (int g = 0; g < MAX_G; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[g][e] = 0.f;
+// ---- exact BF16 rows (the tail, or a whole BF16 cache) on the tensor cores ---------------
+//
+// mma.sync m16n8k16, bf16 x bf16 -> fp32.  Q.K: A = the queries, rows 0..7 the bf16 high
+// part of head g and rows 8..15 the bf16 remainder q - hi (together about 16 significant
+// bits); B = K^T, 8 tokens per n-tile, read straight from the BF16 ring with 16-byte loads:
+// within a 32-channel step s the k order is permuted so that lane (g, tq) supplies channels
+// 32 s + 8 tq + 0..7 of token g; the query fragments follow the same permutation.  The
+// scores of head g, tokens 2tq and 2tq+1 of the n-tile, are the sums of rows g and g+8.
+// P.V: A = the softmax weights (rows g: bf16 high part, rows g+8: remainder), B = V (16
+// tokens x 8 channels) built with byte permutes from four 16-byte row loads; column n of
+// n-tile (j, e) is channel 8 (8 j + n) + e, so a lane's loads are whole 16-byte pieces.  The
+// P.V accumulators stay in fp32 across the whole split (no per-chunk epilogue).
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+
+// (lo, hi) -> bf16x2 with lo in the low half, each rounded to nearest even
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// (x0, x1) split into a bf16x2 high part and a bf16x2 remainder
+__device__ __forceinline__ void bf16_split(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  hi = bf16x2_rn(x0, x1);
+  lo = bf16x2_rn(x0 - bf_lo(hi), x1 - bf_hi(hi));
+}
+
+// Query fragments of the BF16 path for one KV head (all warps of the CTA share them):
+// qfb[ks * 32 + lane] = (a0, a1, a2, a3) of k-step ks = 2 s + h.
+__device__ __forceinline__ void build_qfrag_bf16(uint4 *qfb, const float (*qraw)[D], int tid, int nthreads) {
+  for (int t = tid; t < 8 * 32; t += nthreads) {
+    const int ks = t >> 5, l = t & 31, g = l >> 2, tq = l & 3;
+    const int c = 32 * (ks >> 1) + 8 * tq + 4 * (ks & 1);
+    uint4 f;
+    bf16_split(qraw[g][c], qraw[g][c + 1], f.x, f.y);
+    bf16_split(qraw[g][c + 2], qraw[g][c + 3], f.z, f.w);
+    qfb[t] = f;
   }
-  const __nv_bfloat16 *kbase = ring_row(L, seq, head, 0, 0);
-  const __nv_bfloat16 *vbase = ring_row(L, seq, head, 1, 0);
+}
+
+// Tokens [a + c0*32, a + c1*32) (clipped to b) of one warp: online-softmax state of the
+// 8 head slots written to mw / lw / accw.  Ring rows past b may hold anything: their K and
+// V loads are replaced by zeros and their scores by -inf.
+__device__ __forceinline__ void warp_bf16_tc(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
+                                             int64_t c1, int64_t cdirty, const uint4 *qfb, float *mw, float *lw,
+                                             float *accw) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const uint4 *kbase = reinterpret_cast<const uint4 *>(ring_row(L, seq, head, 0, 0));
+  const uint4 *vbase = reinterpret_cast<const uint4 *>(ring_row(L, seq, head, 1, 0));
+  // ring slots in 32 bits (a ring holds at most max_ctx < 2^31 rows); slot0 advances by one
+  // chunk per iteration
+  const int R = (int)L.ring_cap;
+  int slot0 = (int)((a + c0 * CH) % L.ring_cap);
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  float acc[2][8][4];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[j][e][i] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
 #pragma unroll 1
   for (int64_t ci = c0; ci < c1; ++ci) {
     if (ci == (cdirty > c0 ? cdirty : c0) && cdirty < c1) wait_producer();
     const int64_t i0 = a + ci * CH;
     const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
-    const bool valid = lane < nvalid;
-    const int64_t slot0 = i0 % L.ring_cap;  // ring row of token i0; later rows wrap
-    float sc[MAX_G];
+    // ---- Q.K: 4 n-tiles of 8 tokens; lane row = token 8 nt + g
+    float sc[8];
 #pragma unroll
-    for (int g = 0; g < MAX_G; ++g) sc[g] = 0.f;
-    if (valid) {
-      int64_t sl = slot0 + lane;
-      if (sl >= L.ring_cap) sl -= L.ring_cap;
-      const uint4 *row = reinterpret_cast<const uint4 *>(kbase + sl * D);
-      uint4 raw[D / 8];
+    for (int nt = 0; nt < 4; ++nt) {
+      const int t = 8 * nt + g;
+      int sl = slot0 + t;
+      if (sl >= R) sl -= R;
+      const uint4 *row = kbase + (size_t)sl * (2 * D / 16);
+      uint4 kr[4];
 #pragma unroll
-      for (int j8 = 0; j8 < D / 8; ++j8) raw[j8] = row[j8];
+      for (int s2 = 0; s2 < 4; ++s2) kr[s2] = t < nvalid ? __ldg(row + 4 * s2 + tq) : zero;
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j8 = 0; j8 < D / 8; ++j8) {
-        float x[8];
-        const uint32_t w[4] = {raw[j8].x, raw[j8].y, raw[j8].z, raw[j8].w};
+      for (int s2 = 0; s2 < 4; ++s2) {
+        mma_bf16(d, qfb[(2 * s2) * 32 + lane], kr[s2].x, kr[s2].y);
+        mma_bf16(d, qfb[(2 * s2 + 1) * 32 + lane], kr[s2].z, kr[s2].w);
+      }
+      sc[2 * nt] = 8 * nt + 2 * tq < nvalid ? d[0] + d[2] : -INFINITY;
+      sc[2 * nt + 1] = 8 * nt + 2 * tq + 1 < nvalid ? d[1] + d[3] : -INFINITY;
+    }
+    // ---- online softmax of head g (the 4 lanes tq of a group hold the chunk's 32 tokens)
+    float cmax = sc[0];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          x[2 * u] = __uint_as_float(w[u] << 16);
-          x[2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
-        }
+    for (int k = 1; k < 8; ++k) cmax = fmaxf(cmax, sc[k]);
+    cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 1));
+    cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 2));
+    const float mn = fmaxf(m_run, cmax);  // finite: every chunk holds a valid token
+    const float alpha = exp2_fast(m_run - mn);
+    float p[8], psum = 0.f;
 #pragma unroll
-        for (int g = 0; g < MAX_G; ++g) {
-          if (g >= G) break;
-          const float4 qa = *reinterpret_cast<const float4 *>(&qraw[g][8 * j8]);
-          const float4 qb = *reinterpret_cast<const float4 *>(&qraw[g][8 * j8 + 4]);
-          float t = sc[g];
-          t = fmaf(x[0], qa.x, t);
-          t = fmaf(x[1], qa.y, t);
-          t = fmaf(x[2], qa.z, t);
-          t = fmaf(x[3], qa.w, t);
-          t = fmaf(x[4], qb.x, t);
-          t = fmaf(x[5], qb.y, t);
-          t = fmaf(x[6], qb.z, t);
-          t = fmaf(x[7], qb.w, t);
-          sc[g] = t;
+    for (int k = 0; k < 8; ++k) {
+      p[k] = exp2_fast(sc[k] - mn);
+      psum += p[k];
+    }
+    l_run = l_run * alpha + psum;
+    m_run = mn;
+    if (__any_sync(FULL, alpha != 1.f)) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[j][e][i] *= alpha;
+    }
+    // ---- P.V: 2 k-steps of 16 tokens
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt) {
+      uint4 pa;  // rows g / g+8: weights of tokens 16 kt + 2tq + (0, 1) and 16 kt + 8 + 2tq + (0, 1)
+      bf16_split(p[4 * kt], p[4 * kt + 1], pa.x, pa.y);
+      bf16_split(p[4 * kt + 2], p[4 * kt + 3], pa.z, pa.w);
+      int sl[4];
+      bool vl[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int t = 16 * kt + 2 * tq + (r & 1) + 8 * (r >> 1);
+        vl[r] = t < nvalid;
+        sl[r] = slot0 + t;
+        if (sl[r] >= R) sl[r] -= R;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint4 rv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) rv[r] = vl[r] ? __ldg(vbase + (size_t)sl[r] * (2 * D / 16) + 8 * j + g) : zero;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int w = e >> 1;
+          const unsigned sel = (e & 1) ? 0x7632u : 0x5410u;
+          const uint32_t w0 = w == 0 ? rv[0].x : (w == 1 ? rv[0].y : (w == 2 ? rv[0].z : rv[0].w));
+          const uint32_t w1 = w == 0 ? rv[1].x : (w == 1 ? rv[1].y : (w == 2 ? rv[1].z : rv[1].w));
+          const uint32_t w2 = w == 0 ? rv[2].x : (w == 1 ? rv[2].y : (w == 2 ? rv[2].z : rv[2].w));
+          const uint32_t w3 = w == 0 ? rv[3].x : (w == 1 ? rv[3].y : (w == 2 ? rv[3].z : rv[3].w));
+          mma_bf16(acc[j][e], pa, __byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel));
         }
       }
     }
-#pragma unroll
-    for (int g = 0; g < MAX_G; ++g) {
-      if (g >= G) break;
-      const float sv_ = valid ? sc[g] : -INFINITY;
-      const float mn = fmaxf(m[g], warp_max(sv_));
-      const float alpha = m[g] == -INFINITY ? 0.f : exp2_fast(m[g] - mn);
-      const float p = valid ? exp2_fast(sv_ - mn) : 0.f;
-      l[g] = l[g] * alpha + warp_sum(p);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[g][e] *= alpha;
-      m[g] = mn;
-      pst[lane][g] = p;
-    }
-    __syncwarp();
-    uint2 vr[CH];
-#pragma unroll
-    for (int t = 0; t < CH; ++t) {
-      int64_t sl = slot0 + t;
-      if (sl >= L.ring_cap) sl -= L.ring_cap;
-      vr[t] = t < nvalid ? reinterpret_cast<const uint2 *>(vbase + sl * D)[lane] : make_uint2(0u, 0u);
-    }
-#pragma unroll
-    for (int t = 0; t < CH; ++t) {
-      const float v0 = __uint_as_float(vr[t].x << 16), v1 = __uint_as_float(vr[t].x & 0xffff0000u);
-      const float v2 = __uint_as_float(vr[t].y << 16), v3 = __uint_as_float(vr[t].y & 0xffff0000u);
-      const float4 pa = *reinterpret_cast<const float4 *>(&pst[t][0]);
-      const float4 pb = *reinterpret_cast<const float4 *>(&pst[t][4]);
-      const float pp[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-#pragma unroll
-      for (int g = 0; g < MAX_G; ++g) {
-        if (g >= G) break;
-        acc[g][0] = fmaf(pp[g], v0, acc[g][0]);
-        acc[g][1] = fmaf(pp[g], v1, acc[g][1]);
-        acc[g][2] = fmaf(pp[g], v2, acc[g][2]);
-        acc[g][3] = fmaf(pp[g], v3, acc[g][3]);
-      }
-    }
-    __syncwarp();
+    slot0 += CH;
+    if (slot0 >= R) slot0 -= R;
+  }
+  l_run += __shfl_xor_sync(FULL, l_run, 1);
+  l_run += __shfl_xor_sync(FULL, l_run, 2);
+  if (tq == 0) {
+    mw[g] = m_run;
+    lw[g] = l_run;
   }
 #pragma unroll
-  for (int g = 0; g < MAX_G; ++g) {
-    if (g >= G) break;
-    if (lane == 0) {
-      mw[g] = m[g];
-      lw[g] = l[g];
-    }
+  for (int j = 0; j < 2; ++j)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) accw[g * D + 4 * lane + e] = acc[g][e];
-  }
+    for (int e = 0; e < 8; ++e) {
+      accw[g * D + 8 * (8 * j + 2 * tq) + e] = acc[j][e][0] + acc[j][e][2];
+      accw[g * D + 8 * (8 * j + 2 * tq + 1) + e] = acc[j][e][1] + acc[j][e][3];
+    }
 }
 
 // H.x of one 128-wide row by one warp: the lane holds x[4 lane .. 4 lane + 3]; butterfly
@@ -834,9 +909,16 @@ __host__ __device__ constexpr int warp_area() {
   if constexpr (FAM == FAM_BF16) {
     return 16384;  // accumulators, then (all warps together) the merge's staged partials
   } else {
-    constexpr int s = Stage<FAM, BITS>::NST * Stage<FAM, BITS>::BYTES;
+    // stages, then (kvarn) the page area
+    constexpr int s = Stage<FAM, BITS>::NST * Stage<FAM, BITS>::BYTES + (FAM == FAM_KVARN ? (int)sizeof(PageArea) : 0);
     return s > MAX_G * D * 4 ? s : MAX_G * D * 4;
   }
+}
+
+// the page area of a warp (kvarn): after its stages
+template <int FAM, int BITS>
+__device__ __forceinline__ PageArea *page_area(uint8_t *warp_base) {
+  return reinterpret_cast<PageArea *>(warp_base + Stage<FAM, BITS>::NST * Stage<FAM, BITS>::BYTES);
 }
 
 // [SmemFixed][warp areas]
@@ -888,7 +970,7 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
   if constexpr (FAM != FAM_BF16) {
     if (!tail)
       warp_quant_prefetch<FAM, BITS>(L, s.seq, head, a, (int)c0, (int)c1, cdirty, waited, warp_mem + (size_t)warp * WA,
-                                     lane, pc);
+                                     lane, pc, page_area<FAM, BITS>(warp_mem + (size_t)warp * WA));
   }
   // query rows of this KV head, pre-scaled by softmax_scale * log2(e); heads >= G are 0
   for (int idx = tid; idx < MAX_G * D; idx += DT) {
@@ -900,7 +982,14 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
     F.lw[idx / MAX_G][idx % MAX_G] = 0.f;
   }
   __syncthreads();
-  if (!tail && A.rotk) {
+  // BF16 rows (the tail splits, or a whole BF16 cache) take the raw q as bf16 MMA fragments,
+  // kept in the q' area
+  const bool bf16_rows = tail || FAM == FAM_BF16;
+  uint4 *qfb = reinterpret_cast<uint4 *>(&F.qrot[0][0]);
+  static_assert(sizeof(F.qrot) >= 8 * 32 * sizeof(uint4), "q' area holds the BF16 query fragments");
+  if (bf16_rows) {
+    build_qfrag_bf16(qfb, F.qraw, tid, DT);
+  } else if (A.rotk) {
     // q' = H.q.kappa, one warp per query head
     if (warp < G) {
       float v[4];
@@ -916,22 +1005,14 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
   __syncthreads();
 
   float *accw = reinterpret_cast<float *>(warp_mem + (size_t)warp * WA);  // [MAX_G][D] after the chunks
-  // BF16 warps: softmax weights of a chunk, after the accumulator in the warp area
-  float(*pst)[MAX_G] = reinterpret_cast<float(*)[MAX_G]>(warp_mem + (size_t)warp * WA + MAX_G * D * 4);
-  static_assert(WA >= MAX_G * D * 4 + CH * MAX_G * 4, "warp area holds accumulator and weights");
-  if constexpr (FAM != FAM_BF16) {
-    if (!tail) {
+  static_assert(WA >= MAX_G * D * 4, "warp area holds the accumulator");
+  if (!bf16_rows) {
+    if constexpr (FAM != FAM_BF16)
       warp_quant<FAM, BITS>(L, s.seq, head, a, b, (int)c0, (int)c1, cdirty, waited, G, F.qrot,
-                            warp_mem + (size_t)warp * WA, F.tabs[warp], F.mw[warp], F.lw[warp], accw, pc);
-    } else {
-      for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
-      __syncwarp();
-      warp_bf16(L, s.seq, head, a, b, c0, c1, cdirty, G, F.qraw, pst, F.mw[warp], F.lw[warp], accw);
-    }
+                            warp_mem + (size_t)warp * WA, F.tabs[warp], F.mw[warp], F.lw[warp], accw, pc,
+                            page_area<FAM, BITS>(warp_mem + (size_t)warp * WA));
   } else {
-    for (int idx = lane; idx < MAX_G * D; idx += 32) accw[idx] = 0.f;
-    __syncwarp();
-    warp_bf16(L, s.seq, head, a, b, c0, c1, cdirty, G, F.qraw, pst, F.mw[warp], F.lw[warp], accw);
+    warp_bf16_tc(L, s.seq, head, a, b, c0, c1, cdirty, qfb, F.mw[warp], F.lw[warp], accw);
   }
   __syncthreads();
 
@@ -1117,11 +1198,10 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
   (void)ws_bytes;
   const LayerView L = layer_view(c, layer);
   const int hkv = c->p.n_kv_heads, G = n_q_heads / hkv;
-  // relative cost of one token of a (K+V) head pair: quantized tokens by their bytes; BF16
-  // tail tokens on the CUDA-core path take about 5.5 times as long as a quantized token
-  // (measured: ~20 vs ~108 tokens per microsecond and SM)
+  // relative cost of one token of a (K+V) head pair: quantized tokens by their bytes; a BF16
+  // tail token (tensor-core path, 512 bytes) as about twice a quantized one
   const double tbq = (double)token_bytes(c->fam_k, c->bits_k) + token_bytes(c->fam_v, c->bits_v);
-  const double tbt = 5.5 * tbq;
+  const double tbt = 2.0 * tbq;
   for (size_t base = 0; base < seqs.size(); base += MAXS) {
     const size_t cnt = std::min<size_t>(MAXS, seqs.size() - base);
     DArgs A{};
