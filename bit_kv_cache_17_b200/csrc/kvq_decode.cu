@@ -23,8 +23,6 @@ namespace kvq {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-// warps per CTA (one CTA per SM): 12 where the per-warp stages fit, 8 for 6/8-bit codes
-__host__ __device__ constexpr int nwarps(int fam, int bits) { return (fam != 0 && bits <= 5) ? 12 : 8; }
 constexpr int CH = 32;       // tokens per chunk (one per lane)
 constexpr int MAXSQ = 48;    // max splits over the quantized prefix per (seq, head)
 constexpr int MAXST = 16;    // max splits over the tail per (seq, head)
@@ -342,11 +340,13 @@ __device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head
 }
 
 // Per-warp scale tables of one chunk, built with one token per lane.
+template <int FAM>
 struct ChunkTabs {
+  static constexpr int NM = FAM == FAM_ASYM ? CH : 1;
   float k[CH / 2][4][2];  // K: d * t (kvarn) or d, per token pair, block, token (0 past the end)
-  float v[4][CH];   // V: t * d * QFIX / max over the chunk (per block) -> weights in fixed point
-  float km[CH][4];  // qb_1 K: m + d * 2^(b-1)
-  float vm[CH][4];  // qb_1 V: m + d * 2^(b-1)
+  float v[4][CH];         // V: t * d * QFIX / max over the chunk (per block) -> weights in fixed point
+  float km[NM][4];        // qb_1 K: m + d * 2^(b-1)
+  float vm[NM][4];        // qb_1 V: m + d * 2^(b-1)
 };
 
 
@@ -442,7 +442,7 @@ __device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq,
 template <int FAM, int BITS>
 __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head, int64_t a, int64_t b, int c0,
                                            int c1, int64_t cdirty, bool waited, int G, const float (*qrot)[D],
-                                           uint8_t *stages, ChunkTabs &T, float *mw, float *lw, float *accw,
+                                           uint8_t *stages, ChunkTabs<FAM> &T, float *mw, float *lw, float *accw,
                                            PageCursor &pc, PageArea *pa) {
   using S = Stage<FAM, BITS>;
   const int lane = threadIdx.x & 31;
@@ -532,7 +532,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       }
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) T.v[blk][lane] = tdv[blk] * inv[blk];
-      if (FAM == FAM_ASYM) {
+      if constexpr (FAM == FAM_ASYM) {
         const uint2 mkr = *reinterpret_cast<const uint2 *>(st + S::KM + 8 * lane);
         const uint2 mvr = *reinterpret_cast<const uint2 *>(st + S::VM + 8 * lane);
         const float2 mk01 = __half22float2(*reinterpret_cast<const __half2 *>(&mkr.x));
@@ -568,7 +568,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       }
       float s0, s1;
       upk2(mul2(x, pk2(sigp, sigp)), s0, s1);
-      if (FAM == FAM_ASYM) {
+      if constexpr (FAM == FAM_ASYM) {
         const float4 mA = *reinterpret_cast<const float4 *>(&T.km[t0][0]);
         const float4 mB = *reinterpret_cast<const float4 *>(&T.km[t0 + 1][0]);
         s0 = fmaf(mA.x, qf.qs[0], fmaf(mA.y, qf.qs[1], fmaf(mA.z, qf.qs[2], fmaf(mA.w, qf.qs[3], s0))));
@@ -604,7 +604,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     m_run = mn;
 
     // ---- P.V: weights p * (t d QFIX / max) in 16-bit fixed point, two int8 limbs
-    if (FAM == FAM_ASYM) {
+    if constexpr (FAM == FAM_ASYM) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float4 m4 = *reinterpret_cast<const float4 *>(&T.vm[16 * (k >> 2) + 4 * tq + (k & 3)][0]);
@@ -739,123 +739,139 @@ __device__ __forceinline__ void build_qfrag_bf16(uint4 *qfb, const float (*qraw)
 
 // Tokens [a + c0*32, a + c1*32) (clipped to b) of one warp: online-softmax state of the
 // 8 head slots written to mw / lw / accw.  Ring rows past b may hold anything: their K and
-// V loads are replaced by zeros and their scores by -inf.
+// V loads are replaced by zeros and their scores by -inf.  NJ = 2 accumulates all 128
+// channels in one pass over the tokens; NJ = 1 takes two passes of 64 channels (columns
+// n-tile j = pass), recomputing the identical scores, with half the accumulator registers.
+template <int NJ>
 __device__ __forceinline__ void warp_bf16_tc(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
                                              int64_t c1, int64_t cdirty, const uint4 *qfb, float *mw, float *lw,
                                              float *accw) {
   const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const uint4 *kbase = reinterpret_cast<const uint4 *>(ring_row(L, seq, head, 0, 0));
   const uint4 *vbase = reinterpret_cast<const uint4 *>(ring_row(L, seq, head, 1, 0));
-  // ring slots in 32 bits (a ring holds at most max_ctx < 2^31 rows); slot0 advances by one
-  // chunk per iteration
+  // ring slots in 32 bits (a ring holds at most max_ctx < 2^31 rows)
   const int R = (int)L.ring_cap;
-  int slot0 = (int)((a + c0 * CH) % L.ring_cap);
+  const int slot_a = (int)((a + c0 * CH) % L.ring_cap);
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  float acc[2][8][4];
-#pragma unroll
-  for (int j = 0; j < 2; ++j)
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[j][e][i] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+  bool waited = false;
 #pragma unroll 1
-  for (int64_t ci = c0; ci < c1; ++ci) {
-    if (ci == (cdirty > c0 ? cdirty : c0) && cdirty < c1) wait_producer();
-    const int64_t i0 = a + ci * CH;
-    const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
-    // ---- Q.K: 4 n-tiles of 8 tokens; lane row = token 8 nt + g
-    float sc[8];
+  for (int jp = 0; jp < 2 / NJ; ++jp) {
+    float acc[NJ][8][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int t = 8 * nt + g;
-      int sl = slot0 + t;
-      if (sl >= R) sl -= R;
-      const uint4 *row = kbase + (size_t)sl * (2 * D / 16);
-      uint4 kr[4];
+    for (int j = 0; j < NJ; ++j)
 #pragma unroll
-      for (int s2 = 0; s2 < 4; ++s2) kr[s2] = t < nvalid ? __ldg(row + 4 * s2 + tq) : zero;
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int e = 0; e < 8; ++e)
 #pragma unroll
-      for (int s2 = 0; s2 < 4; ++s2) {
-        mma_bf16(d, qfb[(2 * s2) * 32 + lane], kr[s2].x, kr[s2].y);
-        mma_bf16(d, qfb[(2 * s2 + 1) * 32 + lane], kr[s2].z, kr[s2].w);
+        for (int i = 0; i < 4; ++i) acc[j][e][i] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    int slot0 = slot_a;
+#pragma unroll 1
+    for (int64_t ci = c0; ci < c1; ++ci) {
+      if (!waited && ci >= cdirty) {
+        wait_producer();
+        waited = true;
       }
-      sc[2 * nt] = 8 * nt + 2 * tq < nvalid ? d[0] + d[2] : -INFINITY;
-      sc[2 * nt + 1] = 8 * nt + 2 * tq + 1 < nvalid ? d[1] + d[3] : -INFINITY;
-    }
-    // ---- online softmax of head g (the 4 lanes tq of a group hold the chunk's 32 tokens)
-    float cmax = sc[0];
+      const int64_t i0 = a + ci * CH;
+      const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
+      // ---- Q.K: 4 n-tiles of 8 tokens; lane row = token 8 nt + g
+      float sc[8];
 #pragma unroll
-    for (int k = 1; k < 8; ++k) cmax = fmaxf(cmax, sc[k]);
-    cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 1));
-    cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 2));
-    const float mn = fmaxf(m_run, cmax);  // finite: every chunk holds a valid token
-    const float alpha = exp2_fast(m_run - mn);
-    float p[8], psum = 0.f;
+      for (int nt = 0; nt < 4; ++nt) {
+        const int t = 8 * nt + g;
+        int sl = slot0 + t;
+        if (sl >= R) sl -= R;
+        const uint4 *row = kbase + (size_t)sl * (2 * D / 16);
+        uint4 kr[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      p[k] = exp2_fast(sc[k] - mn);
-      psum += p[k];
-    }
-    l_run = l_run * alpha + psum;
-    m_run = mn;
-    if (__any_sync(FULL, alpha != 1.f)) {
+        for (int s2 = 0; s2 < 4; ++s2) kr[s2] = t < nvalid ? __ldg(row + 4 * s2 + tq) : zero;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[j][e][i] *= alpha;
-    }
-    // ---- P.V: 2 k-steps of 16 tokens
-#pragma unroll
-    for (int kt = 0; kt < 2; ++kt) {
-      uint4 pa;  // rows g / g+8: weights of tokens 16 kt + 2tq + (0, 1) and 16 kt + 8 + 2tq + (0, 1)
-      bf16_split(p[4 * kt], p[4 * kt + 1], pa.x, pa.y);
-      bf16_split(p[4 * kt + 2], p[4 * kt + 3], pa.z, pa.w);
-      int sl[4];
-      bool vl[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int t = 16 * kt + 2 * tq + (r & 1) + 8 * (r >> 1);
-        vl[r] = t < nvalid;
-        sl[r] = slot0 + t;
-        if (sl[r] >= R) sl[r] -= R;
+        for (int s2 = 0; s2 < 4; ++s2) {
+          mma_bf16(d, qfb[(2 * s2) * 32 + lane], kr[s2].x, kr[s2].y);
+          mma_bf16(d, qfb[(2 * s2 + 1) * 32 + lane], kr[s2].z, kr[s2].w);
+        }
+        sc[2 * nt] = 8 * nt + 2 * tq < nvalid ? d[0] + d[2] : -INFINITY;
+        sc[2 * nt + 1] = 8 * nt + 2 * tq + 1 < nvalid ? d[1] + d[3] : -INFINITY;
       }
+      // ---- online softmax of head g (the 4 lanes tq of a group hold the chunk's 32 tokens)
+      float cmax = sc[0];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        uint4 rv[4];
+      for (int k = 1; k < 8; ++k) cmax = fmaxf(cmax, sc[k]);
+      cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 1));
+      cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 2));
+      const float mn = fmaxf(m_run, cmax);  // finite: every chunk holds a valid token
+      const float alpha = exp2_fast(m_run - mn);
+      float p[8], psum = 0.f;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) rv[r] = vl[r] ? __ldg(vbase + (size_t)sl[r] * (2 * D / 16) + 8 * j + g) : zero;
+      for (int k = 0; k < 8; ++k) {
+        p[k] = exp2_fast(sc[k] - mn);
+        psum += p[k];
+      }
+      l_run = l_run * alpha + psum;
+      m_run = mn;
+      if (__any_sync(FULL, alpha != 1.f)) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int w = e >> 1;
-          const unsigned sel = (e & 1) ? 0x7632u : 0x5410u;
-          const uint32_t w0 = w == 0 ? rv[0].x : (w == 1 ? rv[0].y : (w == 2 ? rv[0].z : rv[0].w));
-          const uint32_t w1 = w == 0 ? rv[1].x : (w == 1 ? rv[1].y : (w == 2 ? rv[1].z : rv[1].w));
-          const uint32_t w2 = w == 0 ? rv[2].x : (w == 1 ? rv[2].y : (w == 2 ? rv[2].z : rv[2].w));
-          const uint32_t w3 = w == 0 ? rv[3].x : (w == 1 ? rv[3].y : (w == 2 ? rv[3].z : rv[3].w));
-          mma_bf16(acc[j][e], pa, __byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel));
+        for (int j = 0; j < NJ; ++j)
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[j][e][i] *= alpha;
+      }
+      // ---- P.V: 2 k-steps of 16 tokens
+#pragma unroll
+      for (int kt = 0; kt < 2; ++kt) {
+        uint4 pa;  // rows g / g+8: weights of tokens 16 kt + 2tq + (0, 1) and 16 kt + 8 + 2tq + (0, 1)
+        bf16_split(p[4 * kt], p[4 * kt + 1], pa.x, pa.y);
+        bf16_split(p[4 * kt + 2], p[4 * kt + 3], pa.z, pa.w);
+        int sl[4];
+        bool vl[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int t = 16 * kt + 2 * tq + (r & 1) + 8 * (r >> 1);
+          vl[r] = t < nvalid;
+          sl[r] = slot0 + t;
+          if (sl[r] >= R) sl[r] -= R;
+        }
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const int jc = NJ == 2 ? j : jp;  // channel half of these columns
+          uint4 rv[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            rv[r] = vl[r] ? __ldg(vbase + (size_t)sl[r] * (2 * D / 16) + 8 * jc + g) : zero;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int w = e >> 1;
+            const unsigned sel = (e & 1) ? 0x7632u : 0x5410u;
+            const uint32_t w0 = w == 0 ? rv[0].x : (w == 1 ? rv[0].y : (w == 2 ? rv[0].z : rv[0].w));
+            const uint32_t w1 = w == 0 ? rv[1].x : (w == 1 ? rv[1].y : (w == 2 ? rv[1].z : rv[1].w));
+            const uint32_t w2 = w == 0 ? rv[2].x : (w == 1 ? rv[2].y : (w == 2 ? rv[2].z : rv[2].w));
+            const uint32_t w3 = w == 0 ? rv[3].x : (w == 1 ? rv[3].y : (w == 2 ? rv[3].z : rv[3].w));
+            mma_bf16(acc[j][e], pa, __byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel));
+          }
         }
       }
+      slot0 += CH;
+      if (slot0 >= R) slot0 -= R;
     }
-    slot0 += CH;
-    if (slot0 >= R) slot0 -= R;
-  }
-  l_run += __shfl_xor_sync(FULL, l_run, 1);
-  l_run += __shfl_xor_sync(FULL, l_run, 2);
-  if (tq == 0) {
-    mw[g] = m_run;
-    lw[g] = l_run;
-  }
-#pragma unroll
-  for (int j = 0; j < 2; ++j)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      accw[g * D + 8 * (8 * j + 2 * tq) + e] = acc[j][e][0] + acc[j][e][2];
-      accw[g * D + 8 * (8 * j + 2 * tq + 1) + e] = acc[j][e][1] + acc[j][e][3];
+    if (jp == 2 / NJ - 1) {
+      l_run += __shfl_xor_sync(FULL, l_run, 1);
+      l_run += __shfl_xor_sync(FULL, l_run, 2);
+      if (tq == 0) {
+        mw[g] = m_run;
+        lw[g] = l_run;
+      }
     }
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int jc = NJ == 2 ? j : jp;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        accw[g * D + 8 * (8 * jc + 2 * tq) + e] = acc[j][e][0] + acc[j][e][2];
+        accw[g * D + 8 * (8 * jc + 2 * tq + 1) + e] = acc[j][e][1] + acc[j][e][3];
+      }
+    }
+  }
 }
 
 // H.x of one 128-wide row by one warp: the lane holds x[4 lane .. 4 lane + 3]; butterfly
@@ -889,7 +905,7 @@ __device__ __forceinline__ void warp_wht(float (&v)[4], int lane) {
 
 // Shared memory of the kernel (dynamic): fixed part + per-warp stage area (also used for the
 // warps' accumulators once the chunks are done).
-template <int NW>
+template <int NW, int FAM>
 struct SmemFixed {
   float qraw[MAX_G][D];
   float qrot[MAX_G][D];
@@ -900,7 +916,7 @@ struct SmemFixed {
   float red[MAX_G][D];       // merge: sum over the tail splits (original basis)
   float Ls[MAX_G];
   float Mc[MAX_G], Lc[MAX_G];  // this CTA's combined m and l per head
-  ChunkTabs tabs[NW];
+  ChunkTabs<FAM> tabs[NW];
   int is_last;
 };
 
@@ -922,21 +938,37 @@ __device__ __forceinline__ PageArea *page_area(uint8_t *warp_base) {
 }
 
 // [SmemFixed][warp areas]
+template <int FAM, int BITS, int NW>
+__host__ __device__ constexpr size_t smem_bytes_for() {
+  return ((sizeof(SmemFixed<NW, FAM>) + 127) / 128) * 128 + (size_t)NW * warp_area<FAM, BITS>();
+}
+constexpr size_t kSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
+
+// Warps per CTA (one CTA per SM): 16 where the stages fit (the quantized path runs in 128
+// registers), else 12; 8 for 6- and 8-bit codes (about 200 registers) and for BF16 caches.
+template <int FAM, int BITS>
+__host__ __device__ constexpr int nwarps() {
+  if constexpr (FAM == FAM_BF16 || BITS >= 6)
+    return 8;
+  else
+    return smem_bytes_for<FAM, BITS, 16>() <= kSmemMax ? 16 : 12;
+}
+
 template <int FAM, int BITS>
 __host__ __device__ constexpr size_t smem_fixed_bytes() {
-  return ((sizeof(SmemFixed<nwarps(FAM, BITS)>) + 127) / 128) * 128;
+  return ((sizeof(SmemFixed<nwarps<FAM, BITS>(), FAM>) + 127) / 128) * 128;
 }
 
 template <int FAM, int BITS>
 __host__ __device__ constexpr size_t smem_bytes() {
-  return smem_fixed_bytes<FAM, BITS>() + (size_t)nwarps(FAM, BITS) * warp_area<FAM, BITS>();
+  return smem_bytes_for<FAM, BITS, nwarps<FAM, BITS>()>();
 }
 
 template <int FAM, int BITS>
-__global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView L, DArgs A) {
-  constexpr int NW = nwarps(FAM, BITS), DT = 32 * NW;
+__global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerView L, DArgs A) {
+  constexpr int NW = nwarps<FAM, BITS>(), DT = 32 * NW;
   extern __shared__ __align__(128) uint8_t smem[];
-  SmemFixed<NW> &F = *reinterpret_cast<SmemFixed<NW> *>(smem);
+  SmemFixed<NW, FAM> &F = *reinterpret_cast<SmemFixed<NW, FAM> *>(smem);
   uint8_t *warp_mem = smem + smem_fixed_bytes<FAM, BITS>();
   constexpr int WA = warp_area<FAM, BITS>();
 
@@ -1012,7 +1044,8 @@ __global__ void __launch_bounds__(32 * nwarps(FAM, BITS), 1) k_decode(LayerView 
                             warp_mem + (size_t)warp * WA, F.tabs[warp], F.mw[warp], F.lw[warp], accw, pc,
                             page_area<FAM, BITS>(warp_mem + (size_t)warp * WA));
   } else {
-    warp_bf16_tc(L, s.seq, head, a, b, c0, c1, cdirty, qfb, F.mw[warp], F.lw[warp], accw);
+    // quantized kernels keep their tail warps light on registers: two channel passes
+    warp_bf16_tc<FAM == FAM_BF16 ? 2 : 1>(L, s.seq, head, a, b, c0, c1, cdirty, qfb, F.mw[warp], F.lw[warp], accw);
   }
   __syncthreads();
 
@@ -1150,7 +1183,7 @@ template <int FAM, int BITS>
 cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
   constexpr size_t smem = smem_bytes<FAM, BITS>();
   static_assert(smem <= 232448, "shared memory per CTA");
-  static_assert((nwarps(FAM, BITS) * warp_area<FAM, BITS>()) / (PSTRIDE * 4) >= MAX_G, "merge stage holds a split");
+  static_assert((nwarps<FAM, BITS>() * warp_area<FAM, BITS>()) / (PSTRIDE * 4) >= MAX_G, "merge stage holds a split");
   static bool attr = false;
   if (!attr) {
     const cudaError_t e = cudaFuncSetAttribute(k_decode<FAM, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1160,7 +1193,7 @@ cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)A.ncta);
-  cfg.blockDim = dim3(32 * nwarps(FAM, BITS));
+  cfg.blockDim = dim3(32 * nwarps<FAM, BITS>());
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute la[1];
