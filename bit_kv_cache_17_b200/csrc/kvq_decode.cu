@@ -233,6 +233,22 @@ struct VQuad {
 
 __device__ __forceinline__ float h2f(const __half *p, int i) { return __half2float(p[i]); }
 
+// 1/x by the MUFU unit (about 1 ulp): used only for fixed-point normalizers, where
+// QFIX * rcp(max) keeps every scaled value within 16 bits (QFIX = 32639 leaves the margin)
+__device__ __forceinline__ float rcp_fast(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// max over the warp of a non-negative float (its bits order like unsigned integers)
+__device__ __forceinline__ float warp_max_nonneg(float v) {
+  return __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(v)));
+}
+
+// 16-byte global -> shared copy issued only where pred holds (no branch)
+__device__ __forceinline__ void cp_async16_if(void *dst, const void *src, bool pred);
+
 // 2^x by the MUFU unit (flushes results below 2^-126 to 0: negligible softmax weights)
 __device__ __forceinline__ float exp2_fast(float x) {
   float y;
@@ -252,6 +268,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 // 16-byte global -> shared copy through L2 (no register staging), tracked by commit groups
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16_if(void *dst, const void *src, bool pred) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %2, 0;\n @p cp.async.cg.shared.global [%0], [%1], 16;\n}\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"((int)pred)
+      : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
@@ -335,7 +358,7 @@ __device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head
   cp_async16(st + S::KD + 16 * lane, sb + lay.d);
   if constexpr (FAM == FAM_ASYM) cp_async16(st + S::KM + 16 * lane, sb + lay.m);
   if constexpr (FAM == FAM_KVARN) {
-    if (lane < 8) cp_async16(st + S::KT + 16 * lane, (lane < 4 ? pc.sk : pc.sv) + lay.t + tip0 * 2 + 16 * (lane & 3));
+    cp_async16_if(st + S::KT + 16 * (lane & 7), (lane & 4 ? pc.sv : pc.sk) + lay.t + tip0 * 2 + 16 * (lane & 3), lane < 8);
   }
 }
 
@@ -390,7 +413,7 @@ __device__ __forceinline__ void make_qfrag(QFrag &f, const float (*qrot)[D], con
   }
   amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
-  const float inv = amax > 0.f ? QFIX * __frcp_rn(amax) : 0.f;
+  const float inv = amax > 0.f ? QFIX * rcp_fast(amax) : 0.f;
   f.sigp = amax * SCL;
   // x * inv rounded to an integer by one FFMA with 1.5 * 2^23 + 128: the float's low bytes
   // are (qi + 128) mod 2^16, whose byte 1 is the hi limb and byte 0 (with bit 7 flipped) the lo
@@ -524,10 +547,8 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       float inv[4];
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
-        float mx = tdv[blk];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-        inv[blk] = mx > 0.f ? QFIX * __frcp_rn(mx) : 0.f;
+        const float mx = warp_max_nonneg(tdv[blk]);  // t, d >= 0
+        inv[blk] = mx > 0.f ? QFIX * rcp_fast(mx) : 0.f;
         scl[blk] = mx * SCL;
       }
 #pragma unroll
