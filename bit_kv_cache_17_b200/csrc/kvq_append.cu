@@ -508,28 +508,25 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
       x2p[kp][c] = make_float2(__fmul_rn(x0, x0), __fmul_rn(x1, x1));
     }
   const float fng = (float)ng;
+  // S / ng for a full group (ng = 256) is the exact product with 2^-8: the same rounded value
+  // as the division, at the cost of one multiply
+  const bool full = ng == GROUP;
   // channel index this lane ends with after the recursive-halving reduction
   const int cidx = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
   for (int it = 0; it < iters; ++it) {
-    // channel step: S_j = sum_i x2_ij u_i (chain over this lane's tokens, then the butterfly
-    // 16, 8, 4, 2, 1 across lanes done by recursive halving)
-    float u[8];
-    {
-      const float4 ua = *reinterpret_cast<const float4 *>(&S.uS[lane][0]);
-      const float4 ub = *reinterpret_cast<const float4 *>(&S.uS[lane][4]);
-      u[0] = ua.x; u[1] = ua.y; u[2] = ua.z; u[3] = ua.w;
-      u[4] = ub.x; u[5] = ub.y; u[6] = ub.z; u[7] = ub.w;
-    }
+    // channel step: S_j = sum_i x2_ij u_i.  Each lane chains its even-stride tokens
+    // (l + 64 m) and its odd-stride tokens (l + 64 m + 32) separately, two chains per packed
+    // FMA, adds the two, then the butterfly 16, 8, 4, 2, 1 across lanes (recursive halving)
+    float2 u2[4];  // (u of token l + 64 kp, u of token l + 64 kp + 32)
+#pragma unroll
+    for (int kp = 0; kp < 4; ++kp) u2[kp] = *reinterpret_cast<const float2 *>(&S.uS[lane][2 * kp]);
     float v[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-      float acc = 0.0f;
+      float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int kp = 0; kp < 4; ++kp) {
-        acc = __fmaf_rn(x2p[kp][c].x, u[2 * kp], acc);
-        acc = __fmaf_rn(x2p[kp][c].y, u[2 * kp + 1], acc);
-      }
-      v[c] = acc;
+      for (int kp = 0; kp < 4; ++kp) acc = ffma2(x2p[kp][c], u2[kp], acc);
+      v[c] = __fadd_rn(acc.x, acc.y);
     }
     {  // level 16: keep channels [8 b4, 8 b4 + 8)
       const bool hi = lane & 16;
@@ -566,9 +563,10 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     }
     v[0] = __fadd_rn(v[0], __shfl_xor_sync(FULL, v[0], 1));  // level 1
     if ((lane & 1) == 0) {
-      const float c = v[0] > 0.0f ? __fsqrt_rn(__fdiv_rn(v[0], fng)) : 1.0f;
+      const float mean = full ? __fmul_rn(v[0], 1.0f / GROUP) : __fdiv_rn(v[0], fng);
+      const float c = v[0] > 0.0f ? __fsqrt_rn(mean) : 1.0f;
       S.cS[16 * warp + cidx] = c;
-      S.wS[16 * warp + cidx] = __fdiv_rn(1.0f, __fmul_rn(c, c));
+      S.wS[16 * warp + cidx] = __frcp_rn(__fmul_rn(c, c));  // = RN(1 / c^2)
     }
     __syncwarp();
     // token step: R_i = sum_j x2_ij w_j over this warp's 16 channels (chain in channel order),
@@ -600,9 +598,9 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
       const float a0 = __fadd_rn(p[0], p[4]), a1 = __fadd_rn(p[1], p[5]);
       const float a2 = __fadd_rn(p[2], p[6]), a3 = __fadd_rn(p[3], p[7]);
       const float R = __fadd_rn(__fadd_rn(a0, a2), __fadd_rn(a1, a3));
-      const float t = R > 0.0f ? __fsqrt_rn(__fdiv_rn(R, 128.0f)) : 1.0f;
+      const float t = R > 0.0f ? __fsqrt_rn(__fmul_rn(R, 1.0f / D)) : 1.0f;  // R / 128 exactly
       S.tS[tid] = t;
-      S.uS[tid & 31][tid >> 5] = __fdiv_rn(1.0f, __fmul_rn(t, t));
+      S.uS[tid & 31][tid >> 5] = __frcp_rn(__fmul_rn(t, t));  // = RN(1 / t^2)
     }
     __syncthreads();
   }
@@ -611,12 +609,12 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
   if (tid < D) {
     const __half h = scale_to_half(S.cS[tid]);
     reinterpret_cast<__half *>(sub + lay.c)[tid] = h;
-    S.rc[tid] = __fdiv_rn(1.0f, __half2float(h));
+    S.rc[tid] = __frcp_rn(__half2float(h));
   }
   if (tid < ng) {
     const __half h = scale_to_half(S.tS[tid]);
     reinterpret_cast<__half *>(sub + lay.t)[tid] = h;
-    S.rt[tid] = __fdiv_rn(1.0f, __half2float(h));
+    S.rt[tid] = __frcp_rn(__half2float(h));
   }
   __syncthreads();
 

@@ -168,15 +168,18 @@ void kvqo_wht128_f64(double *v) {
 /* Sinkhorn balancing   [p4] "after the WHT ... Sinkhorn picks a scale per dimension"   */
 /* ------------------------------------------------------------------------------------ */
 
-/* Canonical sum of the n products a[i]*u[i] over the group's tokens: 32 partial sums,
- * partial l chains fmaf over tokens l, l+32, l+64, ... in ascending order from 0.0f;
- * the 32 partials are combined by an xor butterfly with offsets 16, 8, 4, 2, 1. */
+/* Canonical sum of the n products a[i]*u[i] over the group's tokens: 32 partial sums.
+ * Partial l is the sum of two chains, each fmaf in ascending order from 0.0f: one over the
+ * tokens l, l+64, l+128, l+192 and one over l+32, l+96, l+160, l+224 (absent tokens of a
+ * partial group are skipped); the 32 partials are combined by an xor butterfly with
+ * offsets 16, 8, 4, 2, 1. */
 static float sum_over_tokens(const float *x2, int n, int j, const float *u) {
   float p[32], q[32];
   for (int l = 0; l < 32; ++l) {
-    float acc = 0.0f;
-    for (int i = l; i < n; i += 32) acc = fmaf(x2[(size_t)i * D + j], u[i], acc);
-    p[l] = acc;
+    float acc[2] = {0.0f, 0.0f};
+    for (int e = 0; e < 2; ++e)
+      for (int i = l + 32 * e; i < n; i += 64) acc[e] = fmaf(x2[(size_t)i * D + j], u[i], acc[e]);
+    p[l] = acc[0] + acc[1];
   }
   for (int off = 16; off >= 1; off >>= 1) {
     for (int l = 0; l < 32; ++l) q[l] = p[l] + p[l ^ off];
