@@ -1076,7 +1076,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   if (warp < G) {
     const float mw = lane < NW ? F.mw[lane][warp] : -INFINITY;
     const float M = warp_max(mw);
-    const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+    const float f = (mw == -INFINITY) ? 0.f : exp2_fast(mw - M);
     if (lane < NW) F.fw[lane][warp] = f;
     const float lsum = warp_sum(lane < NW ? f * F.lw[lane][warp] : 0.f);
     if (lane == 0) {
@@ -1142,7 +1142,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
     for (int u = 0; u < MAXSPL / 32; ++u) {
       const int k = lane + 32 * u;
       if (k < nspl) {
-        const float f = (mk[u] == -INFINITY) ? 0.f : exp2f(mk[u] - M);
+        const float f = (mk[u] == -INFINITY) ? 0.f : exp2_fast(mk[u] - M);
         F.fw[k][g] = f;
         ls = fmaf(f, k < kb1 ? stage[(k * G + g) * PSTRIDE + 1] : F.fl[k][g], ls);
       }

@@ -198,6 +198,7 @@ class KVCache:
         with torch.cuda.device(self.device):
             self.handle = kvq_cache_create(self.params, self.storage.data_ptr(), self.nbytes)
         self._ws = None
+        self._ws_bytes = {}  # (n_seqs, n_q_heads) -> kvq_workspace_bytes
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -216,7 +217,10 @@ class KVCache:
         kvq_append(self.handle, layer, list(seq_ids), list(n_new), k.data_ptr(), v.data_ptr(), self._stream(stream))
 
     def workspace(self, n_seqs, n_q_heads):
-        nb = kvq_workspace_bytes(self.handle, n_seqs, n_q_heads)
+        key = (n_seqs, n_q_heads)
+        nb = self._ws_bytes.get(key)
+        if nb is None:
+            nb = self._ws_bytes[key] = kvq_workspace_bytes(self.handle, n_seqs, n_q_heads)
         if self._ws is None or self._ws.numel() < nb:
             self._ws = self.torch.empty(max(nb, 256), dtype=self.torch.uint8, device=self.device)
         return self._ws
