@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(256) k_spill_qb(LayerView L, Work W, const __n
     quant_asym<BITS, WHICH>(x, sub, lay, tip, lane);
 }
 
-constexpr int KV_THREADS = 256;
+constexpr int KV_THREADS = 512;  // 16 warps: two threads per row / token, 8 x 8 Sinkhorn tiles
 constexpr int XS = D + 1;  // padded row stride of the fp32 tile in shared memory
 
 struct KvarnSmem {
@@ -233,7 +233,7 @@ struct KvarnSmem {
   float tS[GROUP];      // token scales t
   float cS[D];          // channel scales c
   float wS[D];          // 1/c^2
-  float part[8][GROUP]; // token-sum partials of the 8 channel runs
+  float part[16][GROUP];  // token-sum partials of the 16 runs of 8 channels
   float rc[D];          // 1/fp16(c)
   float rt[GROUP];      // 1/fp16(t)
   uint32_t img[GROUP * 16 * 8 / 4];  // packed code area of the sub-page (up to 8-bit codes)
@@ -293,20 +293,23 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
 constexpr float kTieBound = 0.4998779296875f;  // 0.5 - 2^-13
 
-// Thread-per-token quantization of a balanced group (see k_spill_kvarn, step 4).  The block
-// loop is kept rolled: the kernel is long straight-line code executed once per CTA, so its
-// instruction footprint, not its arithmetic, sets the pace.
+// Quantization of a balanced group (see k_spill_kvarn, step 4): warp w takes tokens
+// 32 (w >> 1) + lane and blocks 2 (w & 1), 2 (w & 1) + 1, so that the lanes of a warp read
+// distinct rows of the tile (conflict-free).  The block loop is kept rolled: its instruction
+// footprint, not its arithmetic, sets the pace.
 template <int BITS, int WHICH>
 __device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const SubLayout &lay, int ng, int tid) {
   constexpr int QMAX = (1 << (BITS - 1)) - 1, QMIN = -(1 << (BITS - 1));
   constexpr int WL = plane_lo(BITS), WH = plane_hi(BITS);
   uint8_t *img = reinterpret_cast<uint8_t *>(S.img);
-  if (tid < ng) {
-    const float rti = S.rt[tid];
-    const float *xr = &S.X[tid * XS];
-    uint32_t dlo = 0u, dhi = 0u;
+  const int tok = 32 * (tid >> 6) + (tid & 31), bhalf = (tid >> 5) & 1;
+  if (tok < ng) {
+    const float rti = S.rt[tok];
+    const float *xr = &S.X[tok * XS];
+    uint32_t dpair = 0u;  // fp16 d of the two blocks
 #pragma unroll 1
-    for (int blk = 0; blk < 4; ++blk) {
+    for (int bb = 0; bb < 2; ++bb) {
+      const int blk = 2 * bhalf + bb;
       // y = (x * rc_j) * rt_i, two roundings, on channel pairs
       f32x2 yp[16];
       float amax = 0.0f;
@@ -321,11 +324,7 @@ __device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const Sub
       const __half dh = sat_half(__fdiv_rn(amax, (float)QMAX));
       const float df = __half2float(dh);
       const unsigned short dbits = __half_as_ushort(dh) & 0x7fffu;
-      const uint32_t dv = (uint32_t)__half_as_ushort(dh) << (16 * (blk & 1));
-      if (blk < 2)
-        dlo |= dv;
-      else
-        dhi |= dv;
+      dpair |= (uint32_t)__half_as_ushort(dh) << (16 * bb);
       uint32_t f[32];  // low BITS bits: the code in two's complement
       // a normal, unsaturated d keeps |y / d| <= QMAX (1 + 2^-11): no clamp needed
       const bool plain = dbits >= 0x0400u && dbits != 0x7bffu;
@@ -367,7 +366,7 @@ __device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const Sub
         const int F = 8 / w;
         if (WHICH == 0) {
           // K: channel 32 blk + 4 jj + k -> byte k of word (jj / F, blk), bits (jj % F) w
-          uint8_t *plane = img + tid * 16 * BITS + (pl == 0 ? 0 : 16 * WL);
+          uint8_t *plane = img + tok * 16 * BITS + (pl == 0 ? 0 : 16 * WL);
 #pragma unroll
           for (int m = 0; m < 8; ++m) {
             if (m >= w) break;
@@ -384,7 +383,7 @@ __device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const Sub
         } else {
           // V: channel 32 blk + e of quad token k -> byte k of word e / F of block blk,
           // bits (e % F) w
-          uint8_t *plane = img + (tid >> 2) * 64 * BITS + (pl == 0 ? 0 : 64 * WL) + 16 * w * blk + (tid & 3);
+          uint8_t *plane = img + (tok >> 2) * 64 * BITS + (pl == 0 ? 0 : 64 * WL) + 16 * w * blk + (tok & 3);
 #pragma unroll
           for (int m = 0; m < 32; ++m) {
             if (m >= 4 * w) break;
@@ -399,7 +398,7 @@ __device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const Sub
         }
       }
     }
-    *reinterpret_cast<uint2 *>(sub + lay.d + tid * 8) = make_uint2(dlo, dhi);
+    *reinterpret_cast<uint32_t *>(sub + lay.d + tok * 8 + 4 * bhalf) = dpair;
   }
   __syncthreads();
   const int nbytes = WHICH == 0 ? ng * 16 * BITS : ((ng + 3) / 4) * 64 * BITS;
@@ -407,7 +406,7 @@ __device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const Sub
     reinterpret_cast<uint4 *>(sub)[p] = reinterpret_cast<const uint4 *>(img)[p];
 }
 
-// One CTA (256 threads) per (kvarn group, head, K or V).  Per sequence, s.a is the first
+// One CTA (512 threads) per (kvarn group, head, K or V).  Per sequence, s.a is the first
 // group the append touches (it may be a partial group that grows) and s.b the quantized
 // length Q(n1) after the append; items enumerate (which, group, head) with which = 0 for the
 // first W.total/2 items when K and V are processed by one launch (W.which == 2).
@@ -447,72 +446,78 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     }
   }
 
-  // 1. each thread rotates one row in registers: BF16 -> fp32, butterfly h = 1..64, x kappa
-  if (tid < ng) {
-    const uint4 *row = reinterpret_cast<const uint4 *>(src_row(L, s, head, which, g0 + tid, in));
-    float r[D];
+  // 1. two threads per row rotate it: thread parity h keeps channels 2i + h.  Stage h = 1 pairs
+  //    (2i, 2i+1), which both threads read from the whole row, and every later stage pairs
+  //    channels of one parity (2i + h, 2(i + d) + h), so each thread runs it alone, two
+  //    butterflies per packed add / sub; then x kappa.
+  {
+    const int row = tid >> 1, h = tid & 1;
+    if (row < ng) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(src_row(L, s, head, which, g0 + row, in));
+      float r[D / 2];  // r[i] = channel 2i + h
 #pragma unroll
-    for (int j8 = 0; j8 < D / 8; ++j8) {
-      const uint4 raw = row[j8];
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      for (int j8 = 0; j8 < D / 8; ++j8) {
+        const uint4 raw = src[j8];
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        r[8 * j8 + 2 * u] = __uint_as_float(w[u] << 16);
-        r[8 * j8 + 2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
+        for (int u = 0; u < 4; ++u) {
+          const float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+          r[4 * j8 + u] = h ? __fsub_rn(x0, x1) : __fadd_rn(x0, x1);
+        }
       }
-    }
-    // stage h = 1 on scalars; stages h = 2..64 pair channels (2i, 2i+1) with (2i+h, 2i+1+h),
-    // two butterflies per packed add / sub
+      f32x2 rp[D / 4];  // (r[2m], r[2m+1])
 #pragma unroll
-    for (int j = 0; j < D; j += 2) {
-      const float x = r[j], y = r[j + 1];
-      r[j] = __fadd_rn(x, y);
-      r[j + 1] = __fsub_rn(x, y);
-    }
-    f32x2 rp[D / 2];
+      for (int m = 0; m < D / 4; ++m) rp[m] = pk2(r[2 * m], r[2 * m + 1]);
+      // stage d = 2 (r index distance 1) on scalars
 #pragma unroll
-    for (int i = 0; i < D / 2; ++i) rp[i] = pk2(r[2 * i], r[2 * i + 1]);
-#pragma unroll
-    for (int hp = 1; hp < D / 2; hp <<= 1) {
-#pragma unroll
-      for (int i = 0; i < D / 2; ++i) {
-        if (i & hp) continue;
-        const f32x2 a = rp[i], b = rp[i + hp];
-        rp[i] = add2(a, b);
-        rp[i + hp] = sub2(a, b);
+      for (int m = 0; m < D / 4; ++m) {
+        float a0, a1;
+        upk2(rp[m], a0, a1);
+        rp[m] = pk2(__fadd_rn(a0, a1), __fsub_rn(a0, a1));
       }
-    }
-    const f32x2 kk = pk2(kKappa(), kKappa());
+      // stages d = 4 .. 64 (distance dp = 1 .. 16 in pairs)
 #pragma unroll
-    for (int i = 0; i < D / 2; ++i) {
-      float a, b;
-      upk2(mul2(rp[i], kk), a, b);
-      S.X[tid * XS + 2 * i] = a;
-      S.X[tid * XS + 2 * i + 1] = b;
+      for (int dp = 1; dp < D / 4; dp <<= 1) {
+#pragma unroll
+        for (int m = 0; m < D / 4; ++m) {
+          if (m & dp) continue;
+          const f32x2 a0 = rp[m], a1 = rp[m + dp];
+          rp[m] = add2(a0, a1);
+          rp[m + dp] = sub2(a0, a1);
+        }
+      }
+      const f32x2 kk = pk2(kKappa(), kKappa());
+#pragma unroll
+      for (int m = 0; m < D / 4; ++m) {
+        float a0, a1;
+        upk2(mul2(rp[m], kk), a0, a1);
+        S.X[row * XS + 4 * m + h] = a0;
+        S.X[row * XS + 4 * m + 2 + h] = a1;
+      }
     }
   }
   if (tid < GROUP) S.uS[tid & 31][tid >> 5] = 1.0f;  // first iteration: t = 1
   __syncthreads();
 
   // 2. Sinkhorn on the squared tile held in registers: thread (warp w, lane l) covers channels
-  //    16w..16w+15 and tokens l + 32k (k = 0..7); rows past the group end square to 0.
-  //    x2p[k/2][c] holds tokens (2(k/2), 2(k/2)+1) of channel c for the packed token sums.
-  float2 x2p[4][16];
+  //    8w..8w+7 and tokens l + 32k (k = 0..7); rows past the group end square to 0.
+  //    x2p[kp][c] holds tokens (l + 64 kp, l + 64 kp + 32) of channel 8w + c.
+  float2 x2p[4][8];
 #pragma unroll
   for (int kp = 0; kp < 4; ++kp)
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const int i0 = lane + 32 * (2 * kp), i1 = lane + 32 * (2 * kp + 1);
-      const float x0 = i0 < ng ? S.X[i0 * XS + 16 * warp + c] : 0.0f;
-      const float x1 = i1 < ng ? S.X[i1 * XS + 16 * warp + c] : 0.0f;
+    for (int c = 0; c < 8; ++c) {
+      const int i0 = lane + 64 * kp, i1 = i0 + 32;
+      const float x0 = i0 < ng ? S.X[i0 * XS + 8 * warp + c] : 0.0f;
+      const float x1 = i1 < ng ? S.X[i1 * XS + 8 * warp + c] : 0.0f;
       x2p[kp][c] = make_float2(__fmul_rn(x0, x0), __fmul_rn(x1, x1));
     }
   const float fng = (float)ng;
   // S / ng for a full group (ng = 256) is the exact product with 2^-8: the same rounded value
   // as the division, at the cost of one multiply
   const bool full = ng == GROUP;
-  // channel index this lane ends with after the recursive-halving reduction
-  const int cidx = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
+  // channel index (within the warp's 8) this lane ends with after the recursive halving
+  const int cidx = 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
   for (int it = 0; it < iters; ++it) {
     // channel step: S_j = sum_i x2_ij u_i.  Each lane chains its even-stride tokens
     // (l + 64 m) and its odd-stride tokens (l + 64 m + 32) separately, two chains per packed
@@ -520,84 +525,75 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     float2 u2[4];  // (u of token l + 64 kp, u of token l + 64 kp + 32)
 #pragma unroll
     for (int kp = 0; kp < 4; ++kp) u2[kp] = *reinterpret_cast<const float2 *>(&S.uS[lane][2 * kp]);
-    float v[16];
+    float v[8];
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 0; c < 8; ++c) {
       float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int kp = 0; kp < 4; ++kp) acc = ffma2(x2p[kp][c], u2[kp], acc);
       v[c] = __fadd_rn(acc.x, acc.y);
     }
-    {  // level 16: keep channels [8 b4, 8 b4 + 8)
+    {  // level 16: keep channels [4 b16, 4 b16 + 4)
       const bool hi = lane & 16;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float send = hi ? v[c] : v[c + 8];
-        const float keep = hi ? v[c + 8] : v[c];
+      for (int c = 0; c < 4; ++c) {
+        const float send = hi ? v[c] : v[c + 4];
+        const float keep = hi ? v[c + 4] : v[c];
         v[c] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 16));
       }
     }
     {  // level 8
       const bool hi = lane & 8;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float send = hi ? v[c] : v[c + 4];
-        const float keep = hi ? v[c + 4] : v[c];
+      for (int c = 0; c < 2; ++c) {
+        const float send = hi ? v[c] : v[c + 2];
+        const float keep = hi ? v[c + 2] : v[c];
         v[c] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 8));
       }
     }
     {  // level 4
       const bool hi = lane & 4;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const float send = hi ? v[c] : v[c + 2];
-        const float keep = hi ? v[c + 2] : v[c];
-        v[c] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 4));
-      }
-    }
-    {  // level 2
-      const bool hi = lane & 2;
       const float send = hi ? v[0] : v[1];
       const float keep = hi ? v[1] : v[0];
-      v[0] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 2));
+      v[0] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, 4));
     }
+    v[0] = __fadd_rn(v[0], __shfl_xor_sync(FULL, v[0], 2));  // level 2
     v[0] = __fadd_rn(v[0], __shfl_xor_sync(FULL, v[0], 1));  // level 1
-    if ((lane & 1) == 0) {
+    if ((lane & 3) == 0) {
       const float mean = full ? __fmul_rn(v[0], 1.0f / GROUP) : __fdiv_rn(v[0], fng);
       const float c = v[0] > 0.0f ? __fsqrt_rn(mean) : 1.0f;
-      S.cS[16 * warp + cidx] = c;
-      S.wS[16 * warp + cidx] = __frcp_rn(__fmul_rn(c, c));  // = RN(1 / c^2)
+      S.cS[8 * warp + cidx] = c;
+      S.wS[8 * warp + cidx] = __frcp_rn(__fmul_rn(c, c));  // = RN(1 / c^2)
     }
     __syncwarp();
-    // token step: R_i = sum_j x2_ij w_j over this warp's 16 channels (chain in channel order),
-    // two tokens per packed FMA
-    float w[16];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const float4 wv = *reinterpret_cast<const float4 *>(&S.wS[16 * warp + 4 * q4]);
-      w[4 * q4] = wv.x; w[4 * q4 + 1] = wv.y; w[4 * q4 + 2] = wv.z; w[4 * q4 + 3] = wv.w;
+    // token step: R_i = sum_j x2_ij w_j; this warp's partial is the chain over its 8 channels
+    // in order, two tokens per packed FMA
+    float w[8];
+    {
+      const float4 wa = *reinterpret_cast<const float4 *>(&S.wS[8 * warp]);
+      const float4 wb = *reinterpret_cast<const float4 *>(&S.wS[8 * warp + 4]);
+      w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
+      w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
     }
-    float2 racc[4];
 #pragma unroll
     for (int kp = 0; kp < 4; ++kp) {
       float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) acc = ffma2(x2p[kp][c], make_float2(w[c], w[c]), acc);
-      racc[kp] = acc;
-    }
-#pragma unroll
-    for (int kp = 0; kp < 4; ++kp) {
-      S.part[warp][lane + 32 * (2 * kp)] = racc[kp].x;
-      S.part[warp][lane + 32 * (2 * kp + 1)] = racc[kp].y;
+      for (int c = 0; c < 8; ++c) acc = ffma2(x2p[kp][c], make_float2(w[c], w[c]), acc);
+      S.part[warp][lane + 64 * kp] = acc.x;
+      S.part[warp][lane + 64 * kp + 32] = acc.y;
     }
     __syncthreads();
     if (tid < ng) {
-      float p[8];
+      // the 16 run partials by the xor butterfly 8, 4, 2, 1
+      float p[16];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) p[r] = S.part[r][tid];
-      const float a0 = __fadd_rn(p[0], p[4]), a1 = __fadd_rn(p[1], p[5]);
-      const float a2 = __fadd_rn(p[2], p[6]), a3 = __fadd_rn(p[3], p[7]);
-      const float R = __fadd_rn(__fadd_rn(a0, a2), __fadd_rn(a1, a3));
+      for (int r = 0; r < 16; ++r) p[r] = S.part[r][tid];
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+        for (int r = 0; r < off; ++r) p[r] = __fadd_rn(p[r], p[r + off]);
+      const float R = p[0];
       const float t = R > 0.0f ? __fsqrt_rn(__fmul_rn(R, 1.0f / D)) : 1.0f;  // R / 128 exactly
       S.tS[tid] = t;
       S.uS[tid & 31][tid >> 5] = __frcp_rn(__fmul_rn(t, t));  // = RN(1 / t^2)

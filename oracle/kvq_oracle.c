@@ -188,18 +188,18 @@ static float sum_over_tokens(const float *x2, int n, int j, const float *u) {
   return p[0];
 }
 
-/* Canonical sum of the 128 products row[j]*w[j] of one token: 8 partial sums, partial r
- * chains fmaf over channels 16r .. 16r+15 in ascending order from 0.0f; the 8 partials
- * are combined by an xor butterfly with offsets 4, 2, 1. */
+/* Canonical sum of the 128 products row[j]*w[j] of one token: 16 partial sums, partial r
+ * chains fmaf over channels 8r .. 8r+7 in ascending order from 0.0f; the 16 partials are
+ * combined by an xor butterfly with offsets 8, 4, 2, 1. */
 static float sum_over_channels(const float *row2, const float *w) {
-  float p[8], q[8];
-  for (int r = 0; r < 8; ++r) {
+  float p[16], q[16];
+  for (int r = 0; r < 16; ++r) {
     float acc = 0.0f;
-    for (int j = 16 * r; j < 16 * r + 16; ++j) acc = fmaf(row2[j], w[j], acc);
+    for (int j = 8 * r; j < 8 * r + 8; ++j) acc = fmaf(row2[j], w[j], acc);
     p[r] = acc;
   }
-  for (int off = 4; off >= 1; off >>= 1) {
-    for (int r = 0; r < 8; ++r) q[r] = p[r] + p[r ^ off];
+  for (int off = 8; off >= 1; off >>= 1) {
+    for (int r = 0; r < 16; ++r) q[r] = p[r] + p[r ^ off];
     memcpy(p, q, sizeof p);
   }
   return p[0];
