@@ -84,3 +84,50 @@ def test_append_decode_64k():
         ref = oracle.decode_head("kvarn4", "kvarn4", cfg["k"][h], cfg["v"][h], tail, q[h * G:(h + 1) * G])
         H.check_decode(got[h * G:(h + 1) * G], ref, f"64k head {h}")
     assert c.status() == 0
+
+
+@pytest.mark.parametrize("type_", ["bf16", "q8_0"])
+def test_append_decode_short_context_and_bf16(type_):
+    """A BF16 cache (every row in the ring: the decode follows the ring-write kernel) and a
+    q8_0 cache whose first steps do not spill (context below the tail)."""
+    th = H.torch()
+    hkv, hq, tail = 2, 8, 64
+    rng = np.random.default_rng(41)
+    k, v, _ = synth.kv_ar1(rng, hkv, 120)
+    c = H.make_cache(type_, hkv, 256, tail if type_ != "bf16" else 0)
+    n = 40
+    c.append(0, [0], [n], H.to_dev_bf16(_rows(k, 0, n)), H.to_dev_bf16(_rows(v, 0, n)))
+    for step in range(4):
+        m = 1 if step < 3 else 30  # the last step crosses the tail and spills
+        q = synth.queries(rng, 1, 1, hq)[0]
+        out = c.append_decode(0, [0], [m], H.to_dev_bf16(_rows(k, n, n + m)), H.to_dev_bf16(_rows(v, n, n + m)),
+                              th.from_numpy(q).cuda())
+        th.cuda.synchronize()
+        n += m
+        _check(c, type_, [(k, v)], [n], tail if type_ != "bf16" else 0, [0], q, out.cpu().numpy().astype(np.float64))
+    assert c.status() == 0
+
+
+def test_append_decode_more_sequences_than_one_launch():
+    """70 sequences: the append and the decode each take two launches (64 sequences per
+    launch), so the decode is not overlapped; every output still matches the oracle."""
+    th = H.torch()
+    hkv, hq, tail, S = 1, 2, 32, 70
+    rng = np.random.default_rng(43)
+    lens = [int(x) for x in rng.integers(1, 200, S)]
+    data = [synth.kv_ar1(rng, hkv, lens[s] + 1)[:2] for s in range(S)]
+    c = H.make_cache("kvarn3", hkv, 256, tail, n_seqs=S)
+    H.append(c, 0, list(range(S)), [(_rows(data[s][0], 0, lens[s]), _rows(data[s][1], 0, lens[s])) for s in range(S)])
+    q = synth.queries(rng, 1, S, hq)[0]
+    ids = list(range(S))[::-1]
+    k = np.concatenate([_rows(data[s][0], lens[s], lens[s] + 1) for s in ids])
+    v = np.concatenate([_rows(data[s][1], lens[s], lens[s] + 1) for s in ids])
+    out = c.append_decode(0, ids, [1] * S, H.to_dev_bf16(k), H.to_dev_bf16(v), th.from_numpy(q).cuda())
+    th.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    for row, s in enumerate(ids):
+        kk, vv = data[s]
+        n = lens[s] + 1
+        ref = H.oracle_decode("kvarn3", kk[:, :n], vv[:, :n], tail, q[row])
+        H.check_decode(got[row], ref, f"seq {s}")
+    assert c.status() == 0
