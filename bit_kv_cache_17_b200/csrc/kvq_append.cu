@@ -560,10 +560,9 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     v[0] = __fadd_rn(v[0], __shfl_xor_sync(FULL, v[0], 2));  // level 2
     v[0] = __fadd_rn(v[0], __shfl_xor_sync(FULL, v[0], 1));  // level 1
     if ((lane & 3) == 0) {
-      const float mean = full ? __fmul_rn(v[0], 1.0f / GROUP) : __fdiv_rn(v[0], fng);
-      const float c = v[0] > 0.0f ? __fsqrt_rn(mean) : 1.0f;
-      S.cS[8 * warp + cidx] = c;
-      S.wS[8 * warp + cidx] = __frcp_rn(__fmul_rn(c, c));  // = RN(1 / c^2)
+      // the iterations carry w_j = 1 / c_j^2 = n / S_j; the scale itself comes from the last S
+      S.cS[8 * warp + cidx] = v[0];
+      S.wS[8 * warp + cidx] = v[0] > 0.0f ? __fdiv_rn(fng, v[0]) : 1.0f;
     }
     __syncwarp();
     // token step: R_i = sum_j x2_ij w_j; this warp's partial is the chain over its 8 channels
@@ -594,21 +593,25 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
 #pragma unroll
         for (int r = 0; r < off; ++r) p[r] = __fadd_rn(p[r], p[r + off]);
       const float R = p[0];
-      const float t = R > 0.0f ? __fsqrt_rn(__fmul_rn(R, 1.0f / D)) : 1.0f;  // R / 128 exactly
-      S.tS[tid] = t;
-      S.uS[tid & 31][tid >> 5] = __frcp_rn(__fmul_rn(t, t));  // = RN(1 / t^2)
+      S.tS[tid] = R;  // u_i = 1 / t_i^2 = 128 / R_i; the scale itself comes from the last R
+      S.uS[tid & 31][tid >> 5] = R > 0.0f ? __fdiv_rn(128.0f, R) : 1.0f;
     }
     __syncthreads();
   }
 
-  // 3. fp16 scales; normalization uses the stored (fp16) values
+  // 3. scales from the last sums, c_j = sqrt(S_j / n) and t_i = sqrt(R_i / 128) (S_j / 256 and
+  //    R_i / 128 are exact products), rounded to fp16; normalization uses the stored values
   if (tid < D) {
-    const __half h = scale_to_half(S.cS[tid]);
+    const float Sj = S.cS[tid];
+    const float c = (iters > 0 && Sj > 0.0f) ? __fsqrt_rn(full ? __fmul_rn(Sj, 1.0f / GROUP) : __fdiv_rn(Sj, fng)) : 1.0f;
+    const __half h = scale_to_half(c);
     reinterpret_cast<__half *>(sub + lay.c)[tid] = h;
     S.rc[tid] = __frcp_rn(__half2float(h));
   }
   if (tid < ng) {
-    const __half h = scale_to_half(S.tS[tid]);
+    const float Ri = S.tS[tid];
+    const float t = (iters > 0 && Ri > 0.0f) ? __fsqrt_rn(__fmul_rn(Ri, 1.0f / D)) : 1.0f;
+    const __half h = scale_to_half(t);
     reinterpret_cast<__half *>(sub + lay.t)[tid] = h;
     S.rt[tid] = __frcp_rn(__half2float(h));
   }

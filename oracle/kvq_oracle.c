@@ -207,26 +207,31 @@ static float sum_over_channels(const float *row2, const float *w) {
 
 /* Scale-only form.  With Y = X / (c_j t_i), the channel step sets
  * c_j = sqrt(mean_i X_ij^2 / t_i^2) and the token step t_i = sqrt(mean_j X_ij^2 / c_j^2);
- * one iteration is a channel step followed by a token step.  A zero sum gives scale 1. */
+ * one iteration is a channel step followed by a token step.  The iterations carry only the
+ * squared reciprocals u_i = 1/t_i^2 = 128 / R_i and w_j = 1/c_j^2 = n / S_j (one division
+ * each, from the sums S_j = sum_i X_ij^2 u_i and R_i = sum_j X_ij^2 w_j); the scales are
+ * taken from the last sums, c_j = sqrt(S_j / n) and t_i = sqrt(R_i / 128).  A zero sum
+ * gives 1 (for the scale and for its reciprocal). */
 void kvqo_sinkhorn(const float *x, int n, int iters, float *c, float *t) {
   float *x2 = (float *)malloc(sizeof(float) * (size_t)n * D);
-  float u[GROUP], w[D];
+  float u[GROUP], w[D], S[D], R[GROUP];
   for (int i = 0; i < n * D; ++i) x2[i] = x[i] * x[i];
-  for (int i = 0; i < n; ++i) t[i] = 1.0f;
-  for (int j = 0; j < D; ++j) c[j] = 1.0f;
+  for (int i = 0; i < n; ++i) u[i] = 1.0f;
   const float fn = (float)n;
+  for (int j = 0; j < D; ++j) S[j] = 0.0f;
+  for (int i = 0; i < n; ++i) R[i] = 0.0f;
   for (int it = 0; it < iters; ++it) {
-    for (int i = 0; i < n; ++i) u[i] = 1.0f / (t[i] * t[i]);
     for (int j = 0; j < D; ++j) {
-      float s = sum_over_tokens(x2, n, j, u);
-      c[j] = s > 0.0f ? sqrtf(s / fn) : 1.0f;
+      S[j] = sum_over_tokens(x2, n, j, u);
+      w[j] = S[j] > 0.0f ? fn / S[j] : 1.0f;
     }
-    for (int j = 0; j < D; ++j) w[j] = 1.0f / (c[j] * c[j]);
     for (int i = 0; i < n; ++i) {
-      float r = sum_over_channels(x2 + (size_t)i * D, w);
-      t[i] = r > 0.0f ? sqrtf(r / 128.0f) : 1.0f;
+      R[i] = sum_over_channels(x2 + (size_t)i * D, w);
+      u[i] = R[i] > 0.0f ? 128.0f / R[i] : 1.0f;
     }
   }
+  for (int j = 0; j < D; ++j) c[j] = (iters > 0 && S[j] > 0.0f) ? sqrtf(S[j] / fn) : 1.0f;
+  for (int i = 0; i < n; ++i) t[i] = (iters > 0 && R[i] > 0.0f) ? sqrtf(R[i] / 128.0f) : 1.0f;
   free(x2);
 }
 
