@@ -66,7 +66,7 @@ size_t plan(kvq_cache *c) {
   c->off_ptab = off;
   off += align_up(sizeof(int32_t) * std::max<int64_t>(1, (int64_t)p.n_seqs * c->max_pages));
   c->off_tickets = off;
-  off += align_up(sizeof(uint32_t) * (size_t)p.n_seqs * p.n_kv_heads);
+  off += align_up(sizeof(uint32_t) * (size_t)std::max<int64_t>(p.n_seqs, kDecodeEntriesPerLaunch) * p.n_kv_heads);
   c->off_status = off;
   off += kAlign;
   c->total = off;
@@ -267,6 +267,32 @@ int kvq_append_decode(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t
   const int budget = info.last_ctas > 0 && info.last_ctas <= c->num_sms / 4 ? c->num_sms - info.last_ctas : 0;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
   return launch_decode(c, layer, dec, n_q_heads, q, scale, out, workspace, ws_bytes, st, budget, pdl);
+}
+
+int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_tokens, int32_t n_q_heads,
+                     const float *q, float softmax_scale, float *out, void *workspace, size_t ws_bytes,
+                     kvq_stream_t stream) {
+  if (!c || layer < 0 || layer >= c->p.n_layers || seq < 0 || seq >= c->p.n_seqs || n_q_tokens < 0)
+    return KVQ_E_INVAL;
+  if (n_q_tokens == 0) return KVQ_OK;
+  if (!q || !out || !workspace || n_q_heads < 1) return KVQ_E_INVAL;
+  if (n_q_heads % c->p.n_kv_heads) return KVQ_E_INVAL;
+  if (n_q_heads / c->p.n_kv_heads > MAX_G) return KVQ_E_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_E_ALIGN;
+  if (ws_bytes < decode_workspace_bytes(c, n_q_tokens, n_q_heads)) return KVQ_E_SIZE;
+  const int64_t n = c->len[(size_t)layer * c->p.n_seqs + seq];
+  if (n_q_tokens > n) return KVQ_E_INVAL;
+  // query i attends to the first n - n_q_tokens + 1 + i tokens of the cache as it is now
+  const int64_t Q = quantized_len(c, n);
+  std::vector<DecodeSeq> entries;
+  entries.reserve(n_q_tokens);
+  for (int i = 0; i < n_q_tokens; ++i) {
+    const int64_t ni = n - n_q_tokens + 1 + i;
+    entries.push_back({seq, i, ni, ni < Q ? ni : Q});
+  }
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
+  return launch_decode(c, layer, entries, n_q_heads, q, scale, out, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,

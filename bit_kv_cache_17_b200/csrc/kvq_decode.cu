@@ -29,7 +29,7 @@ constexpr int MAXST = 16;    // max splits over the tail per (seq, head)
 constexpr int MAXSPL = MAXSQ + MAXST;
 constexpr int PSTRIDE = 4 + D;  // floats per partial: m, l, 2 pad, acc[128] (16-byte records)
 constexpr int PACC = 4;         // offset of acc in a partial
-constexpr int MAXS = 64;        // sequences per launch
+constexpr int MAXS = kDecodeEntriesPerLaunch;  // decode entries (query rows) per launch
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct DSeq {
@@ -133,6 +133,36 @@ __device__ __forceinline__ void mma_s8_fold(f32x2 &x, const uint32_t (&a)[4], ui
       : "+l"(x)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0x4B400000), "l"(bias), "l"(k256),
         "l"(f));
+}
+
+// Q.K of one block with a 24-bit query: the 16-bit part (rows hi / lo as in mma_s8_fold) and a
+// second MMA for the third limb (rows 0..7; rows 8..15 zero), folded as
+//   x += f * (256 * hi + lo + l3 / 254)
+__device__ __forceinline__ void mma_s8_fold3(f32x2 &x, const uint32_t (&a)[4], const uint32_t (&a3)[2], uint32_t b0,
+                                             uint32_t b1, f32x2 f) {
+  const f32x2 bias = 0x4B4000004B400000ull;  // (1.5 * 2^23, 1.5 * 2^23)
+  const f32x2 k256 = 0x4380000043800000ull;  // (256, 256)
+  const f32x2 k254 = 0x3B8102043B810204ull;  // (1/254, 1/254) rounded to fp32
+  asm("{\n"
+      " .reg .b32 c0, c1, c2, c3, e0, e1, e2, e3;\n"
+      " .reg .b64 h, l, m;\n"
+      " mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {c0,c1,c2,c3}, {%1,%2,%3,%4}, {%7,%8}, "
+      "{%9,%9,%9,%9};\n"
+      " mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {e0,e1,e2,e3}, {%5,%13,%6,%13}, {%7,%8}, "
+      "{%9,%9,%9,%9};\n"
+      " mov.b64 h, {c0, c1};\n"
+      " mov.b64 l, {c2, c3};\n"
+      " mov.b64 m, {e0, e1};\n"
+      " sub.rn.f32x2 h, h, %10;\n"
+      " sub.rn.f32x2 l, l, %10;\n"
+      " sub.rn.f32x2 m, m, %10;\n"
+      " fma.rn.f32x2 h, h, %11, l;\n"
+      " fma.rn.f32x2 h, m, %14, h;\n"
+      " fma.rn.f32x2 %0, %12, h, %0;\n"
+      "}\n"
+      : "+l"(x)
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a3[0]), "r"(a3[1]), "r"(b0), "r"(b1), "r"(0x4B400000),
+        "l"(bias), "l"(k256), "l"(f), "r"(0), "l"(k254));
 }
 
 // field s (width W) of each byte of `word`, moved to bits [P, P+W) of the same byte
@@ -379,6 +409,7 @@ struct ChunkTabs {
 // 32 blk + 8 tq + (0..7)).  sigp undoes the fixed point and the codes' byte position.
 struct QFrag {
   uint32_t qa[4][4];
+  uint32_t qa3[4][2];  // third limb: round(254 x the residual of the 16-bit value), rows 0..7
   float sigp;
   float qs[4];  // qb_1: the query summed over each block
 };
@@ -421,12 +452,20 @@ __device__ __forceinline__ void make_qfrag(QFrag &f, const float (*qrot)[D], con
   for (int blk = 0; blk < 4; ++blk) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      uint32_t w[4];
+      uint32_t w[4], z[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) w[i] = __float_as_uint(fmaf(qv[blk * 8 + 4 * h + i], inv, MAGIC));
+      for (int i = 0; i < 4; ++i) {
+        const float xv = qv[blk * 8 + 4 * h + i];
+        const float qsum = fmaf(xv, inv, MAGIC);
+        w[i] = __float_as_uint(qsum);
+        // residual of the rounding, |r| <= 1/2, to 8 more bits: round(254 r) in [-127, 127]
+        const float r = fmaf(xv, inv, MAGIC - qsum);
+        z[i] = __float_as_uint(fmaf(r, 254.0f, MAGIC));
+      }
       const uint32_t x = __byte_perm(w[0], w[1], 0x5140), y = __byte_perm(w[2], w[3], 0x5140);
       f.qa[blk][2 * h] = __byte_perm(x, y, 0x7632);
       f.qa[blk][2 * h + 1] = __byte_perm(x, y, 0x5410) ^ 0x80808080u;
+      f.qa3[blk][h] = __byte_perm(__byte_perm(z[0], z[1], 0x0040), __byte_perm(z[2], z[3], 0x0040), 0x5410) ^ 0x80808080u;
     }
     if constexpr (FAM == FAM_ASYM) {
       float sum = 0.f;
@@ -585,7 +624,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       for (int blk = 0; blk < 4; ++blk) {
         uint32_t b0, b1;
         kt.frag(blk, tq, b0, b1);
-        mma_s8_fold(x, qf.qa[blk], b0, b1, dp[blk]);
+        mma_s8_fold3(x, qf.qa[blk], qf.qa3[blk], b0, b1, dp[blk]);
       }
       float s0, s1;
       upk2(mul2(x, pk2(sigp, sigp)), s0, s1);
@@ -609,10 +648,14 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     // first chunk (m_run = -inf) and the masked tokens
     const float mn = fmaxf(m_run, cmax);
     const float alpha = exp2_fast(m_run - mn);
+    // the weights relative to the chunk's own largest one, pn = 2^(s - cmax) <= 1, so that
+    // their 16-bit fixed point keeps its full range however far the chunk is below the
+    // running max; pm = 2^(cmax - m) scales the chunk back (in l and in the P.V epilogue)
+    const float pm = exp2_fast(cmax - mn);
     float p[8], psum = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      p[k] = exp2_fast(sc[k] - mn);
+      p[k] = exp2_fast(sc[k] - cmax);
       psum += p[k];
     }
     if (__any_sync(FULL, alpha != 1.f)) {
@@ -621,19 +664,22 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) aoff[blk] *= alpha;
     }
-    l_run = l_run * alpha + psum;
+    l_run = fmaf(psum, pm, l_run * alpha);
     m_run = mn;
 
-    // ---- P.V: weights p * (t d QFIX / max) in 16-bit fixed point, two int8 limbs
+    // ---- P.V: weights pn * (t d QFIX / max) in 16-bit fixed point, two int8 limbs
     if constexpr (FAM == FAM_ASYM) {
+      float ao[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float4 m4 = *reinterpret_cast<const float4 *>(&T.vm[16 * (k >> 2) + 4 * tq + (k & 3)][0]);
-        aoff[0] = fmaf(p[k], m4.x, aoff[0]);
-        aoff[1] = fmaf(p[k], m4.y, aoff[1]);
-        aoff[2] = fmaf(p[k], m4.z, aoff[2]);
-        aoff[3] = fmaf(p[k], m4.w, aoff[3]);
+        ao[0] = fmaf(p[k], m4.x, ao[0]);
+        ao[1] = fmaf(p[k], m4.y, ao[1]);
+        ao[2] = fmaf(p[k], m4.z, ao[2]);
+        ao[3] = fmaf(p[k], m4.w, ao[3]);
       }
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) aoff[blk] = fmaf(pm, ao[blk], aoff[blk]);
     }
 #pragma unroll
     for (int blk = 0; blk < 4; ++blk) {
@@ -660,15 +706,17 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
         wa[3] = __byte_perm(x, y, 0x5410) ^ 0x80808080u;
       }
       // per-channel factor of the lane's two columns (channels 8 tq + u and 8 tq + 4 + u of
-      // the block): the block's fixed-point scale, times the page's V channel scale c
+      // the block): the block's fixed-point scale times the chunk factor pm of head g, times
+      // the page's V channel scale c
+      const float sb = scl[blk] * pm;
       f32x2 f[4];
       if (FAM == FAM_KVARN) {
         const f32x2 *cp = reinterpret_cast<const f32x2 *>(&pa->fv[tq][4 * blk]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) f[u] = mul2(pk2(scl[blk], scl[blk]), cp[u]);
+        for (int u = 0; u < 4; ++u) f[u] = mul2(pk2(sb, sb), cp[u]);
       } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) f[u] = pk2(scl[blk], scl[blk]);
+        for (int u = 0; u < 4; ++u) f[u] = pk2(sb, sb);
       }
       VQuad<FAM, BITS> v0, v1;
       v0.load(st + S::VC + tq * S::QS, blk, g);
@@ -965,14 +1013,15 @@ __host__ __device__ constexpr size_t smem_bytes_for() {
 }
 constexpr size_t kSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
 
-// Warps per CTA (one CTA per SM): 16 where the stages fit (the quantized path runs in 128
-// registers), else 12; 8 for 6- and 8-bit codes (about 200 registers) and for BF16 caches.
+// Warps per CTA (one CTA per SM): 12 for codes of up to 5 bits (168 registers: the 24-bit
+// query limbs stay in registers; 16 warps at 128 registers measured no faster), 8 for 6- and
+// 8-bit codes (about 230 registers) and for BF16 caches.
 template <int FAM, int BITS>
 __host__ __device__ constexpr int nwarps() {
   if constexpr (FAM == FAM_BF16 || BITS >= 6)
     return 8;
   else
-    return smem_bytes_for<FAM, BITS, 16>() <= kSmemMax ? 16 : 12;
+    return 12;
 }
 
 template <int FAM, int BITS>
@@ -1103,7 +1152,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const unsigned prev = atomicAdd(&A.tickets[s.seq * A.hkv + head], 1u);
+    const unsigned prev = atomicAdd(&A.tickets[si * A.hkv + head], 1u);
     F.is_last = prev == (unsigned)(nspl - 1);
   }
   __syncthreads();
@@ -1197,7 +1246,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
     o.w = (v[3] + F.red[g][4 * lane + 3]) * inv;
     *reinterpret_cast<float4 *>(A.out + ((int64_t)s.row * A.hkv * G + head * G + g) * D + 4 * lane) = o;
   }
-  if (tid == 0) A.tickets[s.seq * A.hkv + head] = 0u;
+  if (tid == 0) A.tickets[si * A.hkv + head] = 0u;
 }
 
 template <int FAM, int BITS>
@@ -1280,7 +1329,9 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
       nt[i] = d.n > d.Q ? 1 : 0;
       used += hkv * (nq[i] + nt[i]);
     }
-    while (used + hkv <= sms) {
+    // when the entries need more than one wave anyway, plan whole waves
+    const int budget = std::max(sms, ((used + sms - 1) / sms) * sms);
+    while (used + hkv <= budget) {
       int best = -1;
       bool best_t = false;
       double most = 0.0;

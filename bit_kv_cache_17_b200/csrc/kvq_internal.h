@@ -30,6 +30,11 @@ struct kvq_cache {
 
 namespace kvq {
 
+// Decode entries (query rows, each with its own context length) per decode launch; the merge
+// tickets are indexed by (entry within its launch, KV head), so a cache holds this many
+// tickets per head (or n_seqs, if more).
+constexpr int kDecodeEntriesPerLaunch = 64;
+
 // Counts kernel launches (kvq_launch_count).
 void note_launches(int n);
 

@@ -49,6 +49,7 @@ _SIG = {
     "kvq_append": (C.c_int, [_vp, _i32, _i32, C.POINTER(_i32), C.POINTER(_i32), _vp, _vp, _vp]),
     "kvq_workspace_bytes": (C.c_int, [_vp, _i32, _i32, C.POINTER(_sz)]),
     "kvq_decode_attn": (C.c_int, [_vp, _i32, _i32, C.POINTER(_i32), _i32, _vp, C.c_float, _vp, _vp, _sz, _vp]),
+    "kvq_prefill_attn": (C.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, C.c_float, _vp, _vp, _sz, _vp]),
     "kvq_append_decode": (C.c_int, [_vp, _i32, _i32, C.POINTER(_i32), C.POINTER(_i32), _vp, _vp, _i32, _vp,
                                     C.c_float, _vp, _vp, _sz, _vp]),
     "kvq_dequant": (C.c_int, [_vp, _i32, _i32, _i32, _i64, _i64, _i32, _vp, _vp]),
@@ -138,6 +139,12 @@ def kvq_append_decode(h, layer, seq_ids, n_new, k_ptr, v_ptr, n_q_heads, q_ptr, 
     rc = _lib.kvq_append_decode(h, layer, len(seq_ids), _i32arr(seq_ids), _i32arr(n_new), _vp(k_ptr), _vp(v_ptr),
                                 n_q_heads, _vp(q_ptr), softmax_scale, _vp(out_ptr), _vp(ws_ptr), ws_bytes, _vp(stream))
     _check(rc, "kvq_append_decode")
+
+
+def kvq_prefill_attn(h, layer, seq, n_q_tokens, n_q_heads, q_ptr, softmax_scale, out_ptr, ws_ptr, ws_bytes, stream=0):
+    rc = _lib.kvq_prefill_attn(h, layer, seq, n_q_tokens, n_q_heads, _vp(q_ptr), softmax_scale, _vp(out_ptr),
+                               _vp(ws_ptr), ws_bytes, _vp(stream))
+    _check(rc, "kvq_prefill_attn")
 
 
 def kvq_decode_attn_noalloc(h, layer, seq_ids, n_q_heads, q_ptr, softmax_scale, out_ptr, stream=0):
@@ -247,6 +254,18 @@ class KVCache:
         ws = self.workspace(n_seqs, n_q_heads)
         kvq_append_decode(self.handle, layer, list(seq_ids), list(n_new), k.data_ptr(), v.data_ptr(), n_q_heads,
                           q.data_ptr(), softmax_scale, out.data_ptr(), ws.data_ptr(), ws.numel(), self._stream(stream))
+        return out
+
+    def prefill_attn(self, layer, seq, q, out=None, softmax_scale=0.0, stream=None):
+        """kvq_prefill_attn: q [n_q_tokens, n_q_heads, 128] fp32, causal over the chunk of the
+        sequence's newest n_q_tokens tokens."""
+        assert q.dtype == self.torch.float32 and q.is_contiguous()
+        n_q, n_q_heads = q.shape[0], q.shape[1]
+        if out is None:
+            out = self.torch.empty_like(q)
+        ws = self.workspace(n_q, n_q_heads)
+        kvq_prefill_attn(self.handle, layer, seq, n_q, n_q_heads, q.data_ptr(), softmax_scale, out.data_ptr(),
+                         ws.data_ptr(), ws.numel(), self._stream(stream))
         return out
 
     def dequant(self, layer, seq, which, t0, t1, basis=0, out=None, stream=None):

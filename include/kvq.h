@@ -140,6 +140,20 @@ int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *
                     int32_t n_q_heads, const float *q, float softmax_scale, float *out,
                     void *workspace, size_t ws_bytes, kvq_stream_t stream);
 
+/* Attention of a chunk of n_q_tokens queries over the cache of one sequence, causal
+ * within the chunk: query row i attends to the first n - n_q_tokens + 1 + i tokens, n being
+ * the sequence's current length (the chunk's own tokens already appended, as in a prefill
+ * step that writes the chunk's K/V and then attends; the pages' prefill / decode split of
+ * "Fork of beellama and kvarn KV quants at long context").  Every query sees the tokens of
+ * the cache as they are stored now (quantized or BF16 by the current length).
+ * q: device fp32 [n_q_tokens, n_q_heads, 128]; out: device fp32, same shape; softmax_scale
+ * <= 0 selects 1/sqrt(128); workspace: device, >= kvq_workspace_bytes(c, n_q_tokens,
+ * n_q_heads).  KVQ_E_INVAL if n_q_tokens exceeds the sequence length.  Runs the split-K
+ * decode kernel with one entry per query row (64 rows per launch). */
+int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_tokens, int32_t n_q_heads,
+                     const float *q, float softmax_scale, float *out, void *workspace, size_t ws_bytes,
+                     kvq_stream_t stream);
+
 /* One decode step of a layer: kvq_append (n_new[i] tokens to seq_ids[i]) followed by
  * kvq_decode_attn of the same sequences (q / out row i belongs to seq_ids[i]), with the
  * same arguments, layouts and results as the two calls.  The pages ("KV Cache Precision

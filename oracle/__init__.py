@@ -49,6 +49,7 @@ def lib():
             "kvqo_dequant": (_i32, [_i32, _i64, _p, _p, _p, _p, _p, _i32, _p]),
             "kvqo_attend": (None, [_p, _i32, _p, _p, _i64, _f64, _p]),
             "kvqo_decode_head": (_i32, [_i32, _i32, _p, _p, _i64, _i64, _i32, _p, _i32, _f64, _p]),
+            "kvqo_prefill_head": (_i32, [_i32, _i32, _p, _p, _i64, _i64, _i32, _p, _i32, _i32, _f64, _p]),
             "kvqo_payload_bytes": (_f64, [_i32, _i32, _i64, _i64, _i64, _i64, _i64]),
         }
         for name, (res, args) in sig.items():
@@ -235,6 +236,23 @@ def decode_head(type_k, type_v, xk_bf16, xv_bf16, tail, q, scale=None, iters=8):
     out = np.zeros((q.shape[0], D), np.float64)
     r = lib().kvqo_decode_head(_tid(type_k), _tid(type_v), _ptr(xk), _ptr(xv), xk.shape[0], tail, iters,
                                _ptr(q), q.shape[0], float(scale), _ptr(out))
+    assert r == 0
+    return out
+
+
+def prefill_head(type_k, type_v, xk_bf16, xv_bf16, tail, q, scale=None, iters=8):
+    """fp64 attention of a chunk of n_q queries (n_q x G x 128 fp32), the chunk being the n_q
+    newest tokens of one KV head's history: query i sees rows [0, n - n_q + 1 + i) of the
+    state of the full history."""
+    xk = _c(xk_bf16, np.uint16).reshape(-1, D)
+    xv = _c(xv_bf16, np.uint16).reshape(-1, D)
+    q = _c(q, np.float32)
+    n_q, G = q.shape[0], q.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = np.zeros((n_q, G, D), np.float64)
+    r = lib().kvqo_prefill_head(_tid(type_k), _tid(type_v), _ptr(xk), _ptr(xv), xk.shape[0], tail, iters,
+                                _ptr(q), n_q, G, float(scale), _ptr(out))
     assert r == 0
     return out
 

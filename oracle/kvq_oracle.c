@@ -577,6 +577,25 @@ int kvqo_decode_head(int type_k, int type_v, const uint16_t *xk, const uint16_t 
   return rc;
 }
 
+/* Chunk (prefill) reference for one KV head: the stream state of the full n-row history,
+ * then query token i of the chunk (its n_q newest tokens) attends with its G heads to rows
+ * [0, n - n_q + 1 + i) of that state (causal within the chunk). */
+int kvqo_prefill_head(int type_k, int type_v, const uint16_t *xk, const uint16_t *xv, int64_t n, int64_t tail,
+                      int iters, const float *q, int n_q, int G, double scale, double *out) {
+  if (n < 0 || G <= 0 || n_q < 0 || n_q > n) return -1;
+  double *k = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * D);
+  double *v = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * D);
+  double *qd = (double *)malloc(sizeof(double) * (size_t)G * D);
+  int rc = stream_rows(type_k, xk, n, tail, iters, k);
+  if (rc == 0) rc = stream_rows(type_v, xv, n, tail, iters, v);
+  for (int i = 0; rc == 0 && i < n_q; ++i) {
+    for (int j = 0; j < G * D; ++j) qd[j] = (double)q[(size_t)i * G * D + j];
+    kvqo_attend(qd, G, k, v, n - n_q + 1 + i, scale, out + (size_t)i * G * D);
+  }
+  free(k); free(v); free(qd);
+  return rc;
+}
+
 /* ------------------------------------------------------------------------------------ */
 /* size calculator   [p1] "Why the KV cache becomes the bottleneck", "What if the tail  */
 /* grows to 20k"; [p2] "How it works: hybrid storage", "Extended palette"               */

@@ -122,6 +122,13 @@ int kvqo_decode_head(int type_k, int type_v, const uint16_t *x_k_bf16, const uin
                      int64_t n, int64_t tail, int iters, const float *q, int G, double scale,
                      double *out);
 
+/* Chunk (prefill) reference for one KV head: the state of the full n-row history, then query
+ * token i of the chunk (the n_q newest tokens) attends with its G heads to rows
+ * [0, n - n_q + 1 + i) of that state.  q: n_q x G x 128 fp32; out: n_q x G x 128 fp64. */
+int kvqo_prefill_head(int type_k, int type_v, const uint16_t *x_k_bf16, const uint16_t *x_v_bf16,
+                      int64_t n, int64_t tail, int iters, const float *q, int n_q, int G, double scale,
+                      double *out);
+
 /* ---- size calculator ----
  * Payload bytes of a cache of n_layers x n_kv_heads x (K and V) streams of n tokens of
  * head_dim 128 with the newest min(n, tail) tokens kept as 16-bit values.

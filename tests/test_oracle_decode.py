@@ -105,3 +105,33 @@ def test_dequant_rotated_basis_is_rotation_of_original():
     xr = synth.bf16_to_f32(x[:280]).astype(np.float64)
     rel = np.linalg.norm(a - xr) / np.linalg.norm(xr)
     assert rel < 0.1
+
+
+def test_prefill_chunk_reduces_to_decode_and_to_masked_attention():
+    """The chunk reference (query i of the n_q newest tokens sees the first n - n_q + 1 + i
+    rows of the full history's state): with one query it is the decode reference; with BF16
+    rows it is textbook causal attention; with quantized rows it is textbook attention over
+    the prefix of the dequantized state (positions >= Q exact BF16)."""
+    rng = np.random.default_rng(5)
+    n, G, n_q, tail = 700, 3, 9, 200
+    k, v, _ = synth.kv_ar1(rng, 1, n)
+    k, v = k[0], v[0]
+    q = rng.standard_normal((n_q, G, D)).astype(np.float32)
+    scale = 1 / np.sqrt(D)
+    for t in ("kvarn4", "q4_0", "q3_1", "bf16"):
+        tl = tail if t != "bf16" else 0
+        out = oracle.prefill_head(t, t, k, v, tl, q)
+        one = oracle.prefill_head(t, t, k, v, tl, q[-1:])
+        assert np.array_equal(one[0], oracle.decode_head(t, t, k, v, tl, q[-1]))
+        assert np.array_equal(out[-1], one[0])
+        if t == "bf16":
+            kf, vf = synth.bf16_to_f32(k), synth.bf16_to_f32(v)
+        else:
+            st_k, st_v = oracle.stream_state(t, k, tl), oracle.stream_state(t, v, tl)
+            Q = st_k["Q"]
+            kf = np.concatenate([oracle.dequant(t, st_k), synth.bf16_to_f32(k[Q:])])
+            vf = np.concatenate([oracle.dequant(t, st_v), synth.bf16_to_f32(v[Q:])])
+        for i in range(n_q):
+            ni = n - n_q + 1 + i
+            ref = textbook_attention(q[i], kf[:ni], vf[:ni], scale)
+            assert np.max(np.abs(out[i] - ref)) < 1e-10, (t, i)
