@@ -460,6 +460,34 @@ def run_page1_shape(args, kvq, torch, synth):
                         f"tail {tail} (quantized types); layer 0's seeded data in every layer", "per_type": out}
 
 
+def run_prefill(args, kvq, torch, synth):
+    """Chunk attention (kvq_prefill_attn): a 64k-context kvarn4 cache (the headline data) takes
+    a chunk of 16 new tokens, whose 16 queries then attend causally; timed in a CUDA graph
+    cycling layer caches.  One entry per query row: each row reads its whole prefix."""
+    calc = LibCalc(kvq)
+    cfg = synth.config2()
+    n, hkv, hq, tail = cfg["n"], cfg["hkv"], cfg["hq"], cfg["tail"]
+    M, L = 16, 4
+    cache, kt, vt, P = build_decode_workload(torch, kvq, cfg, "kvarn4", L, M)
+    for l in range(L):
+        cache.append(l, [0], [M], kt[P:P + M], vt[P:P + M])
+    q = torch.from_numpy(np.ascontiguousarray(cfg["q"][:M, 0])).cuda()  # [M, hq, 128]
+    o = torch.empty_like(q)
+    cache.workspace(M, hq)
+
+    def fn():
+        for i in range(2 * L):
+            cache.prefill_attn(i % L, 0, q, out=o)
+
+    us = graph_time_us(torch, fn) / (2 * L)
+    b = sum(decode_bytes(calc, "kvarn4", n - M + 1 + i, tail, hkv, 0) for i in range(M)) + 2 * M * hq * D * 4
+    assert cache.status() == 0
+    del cache
+    return {"workload": f"context {n}, kvarn4, tail {tail}, {hkv} KV heads, {hq} query heads, a chunk of {M} "
+                        f"queries (causal)", "us_per_chunk": round(us, 2), "query_rows_per_s": round(M / us * 1e6),
+            "GB_per_s_per_row_reads": round(b / us / 1e3, 1)}
+
+
 def run_quality(args, kvq, torch, synth):
     """Side report (not a target): attention KL(P_bf16 || P_q) and the relative L2 error of the
     attention output of a quantized cache against the BF16 cache of the same data, for every
@@ -707,6 +735,8 @@ def main():
         result["formats_16k"] = run_formats(args, kvq, torch, synth)
         torch.cuda.empty_cache()
         result["page1_shape_240k"] = run_page1_shape(args, kvq, torch, synth)
+        torch.cuda.empty_cache()
+        result["prefill_chunk_64k"] = run_prefill(args, kvq, torch, synth)
         torch.cuda.empty_cache()
         result["quality"] = run_quality(args, kvq, torch, synth)
     if rank == 0 and ws == 1:
