@@ -29,6 +29,31 @@ const char *type_name(int t) {
   return (t >= 0 && t < KVQ_TYPE_COUNT) ? names[t] : "?";
 }
 
+// var_norm: a qb_0 type with the KVarN variance normalization is the kvarn type of the same
+// width (rotation, Sinkhorn, then the symmetric block quantizer); kvarn types already have it.
+int resolve_type(int type, int var_norm, int *out) {
+  const TypeInfo ti = type_info(type);
+  if (ti.fam < 0) return KVQ_E_UNSUPPORTED;
+  *out = type;
+  if (!var_norm || ti.fam == FAM_KVARN) return KVQ_OK;
+  if (ti.fam != FAM_SYM) return KVQ_E_UNSUPPORTED;  // BF16 and the qb_1 types have no such form
+  static const int kvarn_of_bits[9] = {-1, -1, KVQ_KVARN2, KVQ_KVARN3, KVQ_KVARN4, KVQ_KVARN5, KVQ_KVARN6, -1,
+                                       KVQ_KVARN8};
+  *out = kvarn_of_bits[ti.bits];
+  return KVQ_OK;
+}
+
+// Parameters with var_norm applied to the types (the form the cache is planned and built in).
+int resolve_params(const kvq_params *p, kvq_params *r) {
+  if (!p) return KVQ_E_INVAL;
+  if (p->var_norm != 0 && p->var_norm != 1) return KVQ_E_INVAL;
+  *r = *p;
+  int rc = resolve_type(p->type_k, p->var_norm, &r->type_k);
+  if (rc == KVQ_OK) rc = resolve_type(p->type_v, p->var_norm, &r->type_v);
+  r->var_norm = 0;
+  return rc;
+}
+
 int check_params(const kvq_params *p) {
   if (!p) return KVQ_E_INVAL;
   if (p->n_layers < 1 || p->n_seqs < 1 || p->n_kv_heads < 1 || p->max_ctx < 1 || p->tail < 0)
@@ -115,8 +140,12 @@ void kvq_default_params(kvq_params *p) {
   p->page_tokens = GROUP;
 }
 
-int kvq_cache_bytes(const kvq_params *p, size_t *bytes) {
-  int rc = check_params(p);
+int kvq_cache_bytes(const kvq_params *pin, size_t *bytes) {
+  kvq_params rp;
+  int rc = resolve_params(pin, &rp);
+  if (rc) return rc;
+  const kvq_params *p = &rp;
+  rc = check_params(p);
   if (rc) return rc;
   if (!bytes) return KVQ_E_INVAL;
   kvq_cache tmp;
@@ -143,8 +172,12 @@ int kvq_payload_bytes(int32_t type, int32_t raw_bits, int64_t n_layers, int64_t 
   return KVQ_OK;
 }
 
-int kvq_cache_create(const kvq_params *p, void *dev_buf, size_t bytes, kvq_cache **out) {
-  int rc = check_params(p);
+int kvq_cache_create(const kvq_params *pin, void *dev_buf, size_t bytes, kvq_cache **out) {
+  kvq_params rp;
+  int rc = resolve_params(pin, &rp);
+  if (rc) return rc;
+  const kvq_params *p = &rp;
+  rc = check_params(p);
   if (rc) return rc;
   if (!dev_buf || !out) return KVQ_E_INVAL;
   if (!aligned16(dev_buf)) return KVQ_E_ALIGN;

@@ -51,6 +51,18 @@ __device__ __forceinline__ int64_t first_dirty_chunk(int64_t a, int64_t dirty) {
   return dirty <= a ? 0 : (dirty - a) / CH;
 }
 
+// Decode modes.  M_FUSED: Q.K and P.V of one cache type in one kernel.  K and V of different
+// types take two kernels over the same split plan: M_SCORES (the K type) writes the masked
+// Q.K scores of the quantized prefix to the workspace, M_PVEXT (the V type) reads them back
+// for the softmax and P.V (and runs the BF16 tail splits and the merge as M_FUSED does).
+enum DecodeMode { M_FUSED = 0, M_SCORES = 1, M_PVEXT = 2 };
+
+// Where one (entry, KV head) keeps its scores: head slot g at row0 + g * qcap, token i at +i.
+struct ScoreRow {
+  float *row0;
+  int64_t qcap;
+};
+
 struct DArgs {
   int32_t nseq, G, hkv, rotk, rotv, ncta;
   float qscale;  // softmax scale * log2(e)
@@ -58,6 +70,8 @@ struct DArgs {
   float *out;
   float *ws;
   uint32_t *tickets;
+  float *scores;   // M_SCORES / M_PVEXT: [entry][KV head][G][qcap] fp32
+  int64_t qcap;    // tokens per score row (max_ctx rounded up to a chunk)
   DSeq s[MAXS];
 };
 
@@ -355,23 +369,39 @@ struct PageCursor {
 // Copies chunk [i0, i0+32) (K and V codes and fp16 scales; for kvarn, on the first chunk of a
 // page, the page's channel scales) into the stage `st`, 16 bytes per lane and instruction, as
 // one commit group.
-template <int FAM, int BITS>
+template <int FAM, int BITS, int MODE>
 __device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head, int64_t i0, uint8_t *st, int lane,
-                                           PageCursor &pc, PageArea *pa) {
+                                           PageCursor &pc, PageArea *pa, const ScoreRow &sr, int G) {
   using S = Stage<FAM, BITS>;
   const SubLayout lay = sub_layout(FAM, BITS);
   const int64_t page = i0 / GROUP;
+  // the K half (lanes 0..15 for scale pieces) is copied unless the scores come precomputed,
+  // the V half (lanes 16..31) unless only scores are computed
+  constexpr bool KSIDE = MODE != M_PVEXT, VSIDE = MODE != M_SCORES;
+  const bool mine = lane < 16 ? KSIDE : VSIDE;
   if (pc.seek(L, seq, head, page) && FAM == FAM_KVARN)
-    cp_async16(&pa->c[page & 1][lane >> 4][8 * (lane & 15)], (lane < 16 ? pc.sk : pc.sv) + lay.c + 16 * (lane & 15));
+    cp_async16_if(&pa->c[page & 1][lane >> 4][8 * (lane & 15)], (lane < 16 ? pc.sk : pc.sv) + lay.c + 16 * (lane & 15),
+                  mine);
   const int tip0 = (int)(i0 % GROUP);
   constexpr int KP = 32 * BITS;  // 16-byte pieces of K codes (and of V codes)
   constexpr int QP = 4 * BITS;   // pieces per V quad
   // K and V codes of the chunk are contiguous (tip0 is a multiple of 4: V quads are whole)
   const uint8_t *kc = pc.sk + tip0 * 16 * BITS + 16 * lane;
   const uint8_t *vc = pc.sv + tip0 * 16 * BITS + 16 * lane;
+  if constexpr (MODE == M_PVEXT) {
+    // the chunk's scores, head slot g < G: 32 floats = 8 pieces each, into the K code area
 #pragma unroll
-  for (int j = 0; j < KP / 32; ++j) cp_async16(st + S::KC + 16 * lane + 512 * j, kc + 512 * j);
-  if constexpr (32 % QP == 0) {
+    for (int j = 0; j < 2; ++j) {
+      const int p = lane + 32 * j, gg = p >> 3, pc8 = p & 7;
+      cp_async16_if(st + S::KC + 128 * gg + 16 * pc8, sr.row0 + gg * sr.qcap + i0 + 4 * pc8, gg < G);
+    }
+  }
+  if constexpr (KSIDE) {
+#pragma unroll
+    for (int j = 0; j < KP / 32; ++j) cp_async16(st + S::KC + 16 * lane + 512 * j, kc + 512 * j);
+  }
+  if constexpr (!VSIDE) {
+  } else if constexpr (32 % QP == 0) {
     uint8_t *vd = st + S::VC + (lane / QP) * S::QS + 16 * (lane % QP);
 #pragma unroll
     for (int j = 0; j < KP / 32; ++j) cp_async16(vd + j * (32 / QP) * S::QS, vc + 512 * j);
@@ -385,10 +415,12 @@ __device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head
   // fp16 scales: d (and m for qb_1) of K in lanes 0..15, of V in lanes 16..31; t of K in lanes
   // 0..3, of V in lanes 4..7 (kvarn)
   const uint8_t *sb = (lane < 16 ? pc.sk : pc.sv) + tip0 * 8 + 16 * (lane & 15);
-  cp_async16(st + S::KD + 16 * lane, sb + lay.d);
-  if constexpr (FAM == FAM_ASYM) cp_async16(st + S::KM + 16 * lane, sb + lay.m);
+  cp_async16_if(st + S::KD + 16 * lane, sb + lay.d, mine);
+  if constexpr (FAM == FAM_ASYM) cp_async16_if(st + S::KM + 16 * lane, sb + lay.m, mine);
   if constexpr (FAM == FAM_KVARN) {
-    cp_async16_if(st + S::KT + 16 * (lane & 7), (lane & 4 ? pc.sv : pc.sk) + lay.t + tip0 * 2 + 16 * (lane & 3), lane < 8);
+    const bool tmine = (lane & 4) ? VSIDE : KSIDE;
+    cp_async16_if(st + S::KT + 16 * (lane & 7), (lane & 4 ? pc.sv : pc.sk) + lay.t + tip0 * 2 + 16 * (lane & 3),
+                  lane < 8 && tmine);
   }
 }
 
@@ -480,10 +512,10 @@ __device__ __forceinline__ void make_qfrag(QFrag &f, const float (*qrot)[D], con
 
 // Issues the first NST - 1 chunks of a warp's range [c0, c1) (one commit group each, empty
 // groups past the end), so that their copies overlap the query prologue.
-template <int FAM, int BITS>
+template <int FAM, int BITS, int MODE>
 __device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq, int head, int64_t a, int c0, int c1,
                                                     int64_t cdirty, bool &waited, uint8_t *stages, int lane,
-                                                    PageCursor &pc, PageArea *pa) {
+                                                    PageCursor &pc, PageArea *pa, const ScoreRow &sr, int G) {
   using S = Stage<FAM, BITS>;
 #pragma unroll
   for (int j = 0; j < S::NST - 1; ++j) {
@@ -492,7 +524,8 @@ __device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq,
         wait_producer();
         waited = true;
       }
-      copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)(c0 + j) * CH, stages + j * S::BYTES, lane, pc, pa);
+      copy_chunk<FAM, BITS, MODE>(L, seq, head, a + (int64_t)(c0 + j) * CH, stages + j * S::BYTES, lane, pc, pa, sr,
+                                  G);
     }
     cp_async_commit();
   }
@@ -500,13 +533,16 @@ __device__ __forceinline__ void warp_quant_prefetch(const LayerView &L, int seq,
 
 // Q.K and P.V of one warp over its chunks [c0, c1) of a quantized split [a, b) (consecutive, so
 // pages change rarely).  Writes the warp's online-softmax state (m, l and the accumulator in the
-// stored basis) of its heads to shared memory.
-template <int FAM, int BITS>
+// stored basis) of its heads to shared memory.  M_SCORES stops after Q.K and writes the scores
+// to sr instead; M_PVEXT reads them from sr in place of Q.K.
+template <int FAM, int BITS, int MODE>
 __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head, int64_t a, int64_t b, int c0,
                                            int c1, int64_t cdirty, bool waited, int G, const float (*qrot)[D],
                                            uint8_t *stages, ChunkTabs<FAM> &T, float *mw, float *lw, float *accw,
-                                           PageCursor &pc, PageArea *pa) {
+                                           PageCursor &pc, PageArea *pa, const ScoreRow &sr) {
   using S = Stage<FAM, BITS>;
+  constexpr bool KSIDE = MODE != M_PVEXT, VSIDE = MODE != M_SCORES;
+  static_assert(S::KC + MAX_G * CH * 4 <= S::VC || MODE != M_PVEXT, "the K code area holds a chunk's scores");
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   const bool hv = g < G;
@@ -533,7 +569,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
           wait_producer();
           waited = true;
         }
-        copy_chunk<FAM, BITS>(L, seq, head, a + (int64_t)cn * CH, stages + sn * S::BYTES, lane, pc, pa);
+        copy_chunk<FAM, BITS, MODE>(L, seq, head, a + (int64_t)cn * CH, stages + sn * S::BYTES, lane, pc, pa, sr, G);
       }
       cp_async_commit();
       cp_async_wait<S::NST - 1>();  // chunk c has landed (for this lane's copies)
@@ -545,8 +581,8 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       const int nvalid = (int)((b - i0) < CH ? (b - i0) : CH);
       if (page != cur_page && (FAM == FAM_KVARN || cur_page < 0)) {
         const __half *ck = FAM == FAM_KVARN ? pa->c[page & 1][0] : nullptr;
-        make_qfrag<FAM, BITS>(qf, qrot, ck, g, tq, hv);
-        if constexpr (FAM == FAM_KVARN) {
+        if constexpr (KSIDE) make_qfrag<FAM, BITS>(qf, qrot, ck, g, tq, hv);
+        if constexpr (FAM == FAM_KVARN && VSIDE) {
           // lane l builds pairs 2 (l >> 2) and 2 (l >> 2) + 1 of column set tq' = l & 3
           const __half *cv = pa->c[page & 1][1];
           const int tl = lane & 3;
@@ -565,46 +601,49 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     float scl[4];
     {
       const bool vl = lane < nvalid;
-      const uint2 dkr = *reinterpret_cast<const uint2 *>(st + S::KD + 8 * lane);
-      const uint2 dvr = *reinterpret_cast<const uint2 *>(st + S::VD + 8 * lane);
-      const float2 dk01 = __half22float2(*reinterpret_cast<const __half2 *>(&dkr.x));
-      const float2 dk23 = __half22float2(*reinterpret_cast<const __half2 *>(&dkr.y));
-      const float2 dv01 = __half22float2(*reinterpret_cast<const __half2 *>(&dvr.x));
-      const float2 dv23 = __half22float2(*reinterpret_cast<const __half2 *>(&dvr.y));
-      float tkl = 1.f, tvl = 1.f;
-      if (FAM == FAM_KVARN) {
-        tkl = h2f(reinterpret_cast<const __half *>(st + S::KT), lane);
-        tvl = h2f(reinterpret_cast<const __half *>(st + S::VT), lane);
+      if constexpr (KSIDE) {
+        const uint2 dkr = *reinterpret_cast<const uint2 *>(st + S::KD + 8 * lane);
+        const float2 dk01 = __half22float2(*reinterpret_cast<const __half2 *>(&dkr.x));
+        const float2 dk23 = __half22float2(*reinterpret_cast<const __half2 *>(&dkr.y));
+        const float tkl = FAM == FAM_KVARN ? h2f(reinterpret_cast<const __half *>(st + S::KT), lane) : 1.f;
+        // select (not multiply) so that NaN bit patterns in stale rows cannot leak
+        const float dkt[4] = {vl ? dk01.x * tkl : 0.f, vl ? dk01.y * tkl : 0.f, vl ? dk23.x * tkl : 0.f,
+                              vl ? dk23.y * tkl : 0.f};
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) T.k[lane >> 1][blk][lane & 1] = dkt[blk];
+        if constexpr (FAM == FAM_ASYM) {
+          const uint2 mkr = *reinterpret_cast<const uint2 *>(st + S::KM + 8 * lane);
+          const float2 mk01 = __half22float2(*reinterpret_cast<const __half2 *>(&mkr.x));
+          const float2 mk23 = __half22float2(*reinterpret_cast<const __half2 *>(&mkr.y));
+          *reinterpret_cast<float4 *>(&T.km[lane][0]) =
+              make_float4(vl ? fmaf(dk01.x, HALF_RANGE, mk01.x) : 0.f, vl ? fmaf(dk01.y, HALF_RANGE, mk01.y) : 0.f,
+                          vl ? fmaf(dk23.x, HALF_RANGE, mk23.x) : 0.f, vl ? fmaf(dk23.y, HALF_RANGE, mk23.y) : 0.f);
+        }
       }
-      // select (not multiply) so that NaN bit patterns in stale rows cannot leak
-      const float dkt[4] = {vl ? dk01.x * tkl : 0.f, vl ? dk01.y * tkl : 0.f, vl ? dk23.x * tkl : 0.f,
-                            vl ? dk23.y * tkl : 0.f};
+      if constexpr (VSIDE) {
+        const uint2 dvr = *reinterpret_cast<const uint2 *>(st + S::VD + 8 * lane);
+        const float2 dv01 = __half22float2(*reinterpret_cast<const __half2 *>(&dvr.x));
+        const float2 dv23 = __half22float2(*reinterpret_cast<const __half2 *>(&dvr.y));
+        const float tvl = FAM == FAM_KVARN ? h2f(reinterpret_cast<const __half *>(st + S::VT), lane) : 1.f;
+        float tdv[4] = {vl ? dv01.x * tvl : 0.f, vl ? dv01.y * tvl : 0.f, vl ? dv23.x * tvl : 0.f,
+                        vl ? dv23.y * tvl : 0.f};
+        float inv[4];
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) T.k[lane >> 1][blk][lane & 1] = dkt[blk];
-      float tdv[4] = {vl ? dv01.x * tvl : 0.f, vl ? dv01.y * tvl : 0.f, vl ? dv23.x * tvl : 0.f,
-                      vl ? dv23.y * tvl : 0.f};
-      float inv[4];
+        for (int blk = 0; blk < 4; ++blk) {
+          const float mx = warp_max_nonneg(tdv[blk]);  // t, d >= 0
+          inv[blk] = mx > 0.f ? QFIX * rcp_fast(mx) : 0.f;
+          scl[blk] = mx * SCL;
+        }
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        const float mx = warp_max_nonneg(tdv[blk]);  // t, d >= 0
-        inv[blk] = mx > 0.f ? QFIX * rcp_fast(mx) : 0.f;
-        scl[blk] = mx * SCL;
-      }
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) T.v[blk][lane] = tdv[blk] * inv[blk];
-      if constexpr (FAM == FAM_ASYM) {
-        const uint2 mkr = *reinterpret_cast<const uint2 *>(st + S::KM + 8 * lane);
-        const uint2 mvr = *reinterpret_cast<const uint2 *>(st + S::VM + 8 * lane);
-        const float2 mk01 = __half22float2(*reinterpret_cast<const __half2 *>(&mkr.x));
-        const float2 mk23 = __half22float2(*reinterpret_cast<const __half2 *>(&mkr.y));
-        const float2 mv01 = __half22float2(*reinterpret_cast<const __half2 *>(&mvr.x));
-        const float2 mv23 = __half22float2(*reinterpret_cast<const __half2 *>(&mvr.y));
-        *reinterpret_cast<float4 *>(&T.km[lane][0]) =
-            make_float4(vl ? fmaf(dk01.x, HALF_RANGE, mk01.x) : 0.f, vl ? fmaf(dk01.y, HALF_RANGE, mk01.y) : 0.f,
-                        vl ? fmaf(dk23.x, HALF_RANGE, mk23.x) : 0.f, vl ? fmaf(dk23.y, HALF_RANGE, mk23.y) : 0.f);
-        *reinterpret_cast<float4 *>(&T.vm[lane][0]) =
-            make_float4(vl ? fmaf(dv01.x, HALF_RANGE, mv01.x) : 0.f, vl ? fmaf(dv01.y, HALF_RANGE, mv01.y) : 0.f,
-                        vl ? fmaf(dv23.x, HALF_RANGE, mv23.x) : 0.f, vl ? fmaf(dv23.y, HALF_RANGE, mv23.y) : 0.f);
+        for (int blk = 0; blk < 4; ++blk) T.v[blk][lane] = tdv[blk] * inv[blk];
+        if constexpr (FAM == FAM_ASYM) {
+          const uint2 mvr = *reinterpret_cast<const uint2 *>(st + S::VM + 8 * lane);
+          const float2 mv01 = __half22float2(*reinterpret_cast<const __half2 *>(&mvr.x));
+          const float2 mv23 = __half22float2(*reinterpret_cast<const __half2 *>(&mvr.y));
+          *reinterpret_cast<float4 *>(&T.vm[lane][0]) =
+              make_float4(vl ? fmaf(dv01.x, HALF_RANGE, mv01.x) : 0.f, vl ? fmaf(dv01.y, HALF_RANGE, mv01.y) : 0.f,
+                          vl ? fmaf(dv23.x, HALF_RANGE, mv23.x) : 0.f, vl ? fmaf(dv23.y, HALF_RANGE, mv23.y) : 0.f);
+        }
       }
       __syncwarp();
     }
@@ -612,6 +651,16 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
     // ---- Q.K: n-tile r, column n holds token 16(r>>1) + 4(n>>1) + 2(r&1) + (n&1), so that
     //      the lane ends with the scores of tokens 4tq+(0..3) and 16+4tq+(0..3)
     float sc[8];
+    if constexpr (MODE == M_PVEXT) {
+      // the stored scores of head g (0 for the empty head slots), tokens 4tq+(0..3) and 16+4tq+(0..3)
+      const float *sg = reinterpret_cast<const float *>(st + S::KC) + g * CH;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 s0 = hv ? *reinterpret_cast<const float4 *>(sg + 4 * tq) : z;
+      const float4 s1 = hv ? *reinterpret_cast<const float4 *>(sg + 16 + 4 * tq) : z;
+      const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sc[k] = 16 * (k >> 2) + 4 * tq + (k & 3) < nvalid ? sv[k] : -INFINITY;
+    } else {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       KTok<FAM, BITS> kt;
@@ -636,6 +685,16 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
       }
       sc[2 * r] = t0 < nvalid ? s0 : -INFINITY;
       sc[2 * r + 1] = t0 + 1 < nvalid ? s1 : -INFINITY;
+    }
+    }
+    if constexpr (MODE == M_SCORES) {
+      if (hv) {
+        float *dst = sr.row0 + g * sr.qcap + i0 + 4 * tq;
+        *reinterpret_cast<float4 *>(dst) = make_float4(sc[0], sc[1], sc[2], sc[3]);
+        *reinterpret_cast<float4 *>(dst + 16) = make_float4(sc[4], sc[5], sc[6], sc[7]);
+      }
+      __syncwarp();  // every lane is done with this stage before it is refilled next round
+      continue;
     }
 
     // ---- online softmax (head g; the 4 lanes of a group hold the chunk's 32 tokens)
@@ -733,6 +792,7 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
   }
   cp_async_wait<0>();
   __syncwarp();
+  if constexpr (MODE == M_SCORES) return;
   l_run += __shfl_xor_sync(FULL, l_run, 1);
   l_run += __shfl_xor_sync(FULL, l_run, 2);
   if (FAM == FAM_ASYM) {
@@ -1034,8 +1094,9 @@ __host__ __device__ constexpr size_t smem_bytes() {
   return smem_bytes_for<FAM, BITS, nwarps<FAM, BITS>()>();
 }
 
-template <int FAM, int BITS>
+template <int FAM, int BITS, int MODE>
 __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerView L, DArgs A) {
+  static_assert(MODE == M_FUSED || FAM != FAM_BF16, "the score modes take quantized types");
   constexpr int NW = nwarps<FAM, BITS>(), DT = 32 * NW;
   extern __shared__ __align__(128) uint8_t smem[];
   SmemFixed<NW, FAM> &F = *reinterpret_cast<SmemFixed<NW, FAM> *>(smem);
@@ -1052,6 +1113,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   const int head = local / nspl, sp = local % nspl;
   const int G = A.G;
   const bool tail = sp >= s.nsq;
+  if (MODE == M_SCORES && tail) return;  // the BF16 tail splits belong to the P.V kernel
   int64_t a, b;
   int64_t nch;
   if (!tail) {
@@ -1069,10 +1131,12 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   const int64_t cdirty = first_dirty_chunk(a, (tail || FAM == FAM_BF16) ? s.dt : s.dq);
   bool waited = false;
   PageCursor pc;
+  const ScoreRow sr{A.scores + (int64_t)(si * A.hkv + head) * G * A.qcap, A.qcap};
   if constexpr (FAM != FAM_BF16) {
     if (!tail)
-      warp_quant_prefetch<FAM, BITS>(L, s.seq, head, a, (int)c0, (int)c1, cdirty, waited, warp_mem + (size_t)warp * WA,
-                                     lane, pc, page_area<FAM, BITS>(warp_mem + (size_t)warp * WA));
+      warp_quant_prefetch<FAM, BITS, MODE>(L, s.seq, head, a, (int)c0, (int)c1, cdirty, waited,
+                                           warp_mem + (size_t)warp * WA, lane, pc,
+                                           page_area<FAM, BITS>(warp_mem + (size_t)warp * WA), sr, G);
   }
   // query rows of this KV head, pre-scaled by softmax_scale * log2(e); heads >= G are 0
   for (int idx = tid; idx < MAX_G * D; idx += DT) {
@@ -1091,6 +1155,8 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   static_assert(sizeof(F.qrot) >= 8 * 32 * sizeof(uint4), "q' area holds the BF16 query fragments");
   if (bf16_rows) {
     build_qfrag_bf16(qfb, F.qraw, tid, DT);
+  } else if (MODE == M_PVEXT) {
+    // the scores are given: no query on the quantized splits
   } else if (A.rotk) {
     // q' = H.q.kappa, one warp per query head
     if (warp < G) {
@@ -1110,9 +1176,10 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   static_assert(WA >= MAX_G * D * 4, "warp area holds the accumulator");
   if (!bf16_rows) {
     if constexpr (FAM != FAM_BF16)
-      warp_quant<FAM, BITS>(L, s.seq, head, a, b, (int)c0, (int)c1, cdirty, waited, G, F.qrot,
-                            warp_mem + (size_t)warp * WA, F.tabs[warp], F.mw[warp], F.lw[warp], accw, pc,
-                            page_area<FAM, BITS>(warp_mem + (size_t)warp * WA));
+      warp_quant<FAM, BITS, MODE>(L, s.seq, head, a, b, (int)c0, (int)c1, cdirty, waited, G, F.qrot,
+                                  warp_mem + (size_t)warp * WA, F.tabs[warp], F.mw[warp], F.lw[warp], accw, pc,
+                                  page_area<FAM, BITS>(warp_mem + (size_t)warp * WA), sr);
+    if constexpr (MODE == M_SCORES) return;  // every CTA of this kernel is a quantized split
   } else {
     // quantized kernels keep their tail warps light on registers: two channel passes
     warp_bf16_tc<FAM == FAM_BF16 ? 2 : 1>(L, s.seq, head, a, b, c0, c1, cdirty, qfb, F.mw[warp], F.lw[warp], accw);
@@ -1249,14 +1316,14 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   if (tid == 0) A.tickets[si * A.hkv + head] = 0u;
 }
 
-template <int FAM, int BITS>
+template <int FAM, int BITS, int MODE>
 cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
   constexpr size_t smem = smem_bytes<FAM, BITS>();
   static_assert(smem <= 232448, "shared memory per CTA");
   static_assert((nwarps<FAM, BITS>() * warp_area<FAM, BITS>()) / (PSTRIDE * 4) >= MAX_G, "merge stage holds a split");
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(k_decode<FAM, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(k_decode<FAM, BITS, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
@@ -1271,13 +1338,13 @@ cudaError_t run(const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
   la[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = la;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_decode<FAM, BITS>, L, A);
+  return cudaLaunchKernelEx(&cfg, k_decode<FAM, BITS, MODE>, L, A);
 }
 
-cudaError_t dispatch(int fam, int bits, const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
+template <int MODE>
+cudaError_t dispatch_q(int fam, int bits, const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
 #define KVQ_D(F, B) \
-  if (fam == F && bits == B) return run<F, B>(L, A, st, pdl);
-  KVQ_D(FAM_BF16, 16)
+  if (fam == F && bits == B) return run<F, B, MODE>(L, A, st, pdl);
   KVQ_D(FAM_SYM, 2) KVQ_D(FAM_SYM, 3) KVQ_D(FAM_SYM, 4) KVQ_D(FAM_SYM, 5) KVQ_D(FAM_SYM, 6) KVQ_D(FAM_SYM, 8)
   KVQ_D(FAM_ASYM, 2) KVQ_D(FAM_ASYM, 3) KVQ_D(FAM_ASYM, 4) KVQ_D(FAM_ASYM, 5) KVQ_D(FAM_ASYM, 6)
   KVQ_D(FAM_KVARN, 2) KVQ_D(FAM_KVARN, 3) KVQ_D(FAM_KVARN, 4) KVQ_D(FAM_KVARN, 5) KVQ_D(FAM_KVARN, 6)
@@ -1286,18 +1353,41 @@ cudaError_t dispatch(int fam, int bits, const LayerView &L, const DArgs &A, cuda
   return cudaErrorInvalidValue;
 }
 
+cudaError_t dispatch(int fam, int bits, int mode, const LayerView &L, const DArgs &A, cudaStream_t st, bool pdl) {
+  if (mode == M_FUSED && fam == FAM_BF16 && bits == 16) return run<FAM_BF16, 16, M_FUSED>(L, A, st, pdl);
+  if (mode == M_FUSED) return dispatch_q<M_FUSED>(fam, bits, L, A, st, pdl);
+  if (mode == M_SCORES) return dispatch_q<M_SCORES>(fam, bits, L, A, st, pdl);
+  if (mode == M_PVEXT) return dispatch_q<M_PVEXT>(fam, bits, L, A, st, pdl);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
-size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads) {
+// The split partials; for K and V of different types also the scores of the quantized
+// prefix, [entry of a launch][KV head][G][qcap] fp32 after the partials (16-byte aligned).
+size_t decode_partials_bytes(const kvq_cache *c, int n_seqs, int n_q_heads) {
   const int G = n_q_heads / c->p.n_kv_heads;
   return sizeof(float) * (size_t)std::max(n_seqs, 1) * c->p.n_kv_heads * MAXSPL * G * PSTRIDE;
+}
+int64_t decode_score_cap(const kvq_cache *c) { return (c->p.max_ctx + CH - 1) / CH * CH; }
+
+size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads) {
+  const size_t part = decode_partials_bytes(c, n_seqs, n_q_heads);
+  if (c->p.type_k == c->p.type_v) return part;
+  const int G = n_q_heads / c->p.n_kv_heads;
+  const size_t entries = (size_t)std::min(std::max(n_seqs, 1), MAXS);
+  return part + sizeof(float) * entries * c->p.n_kv_heads * G * (size_t)decode_score_cap(c);
 }
 
 int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &seqs, int n_q_heads,
                   const float *q, float scale, float *out, void *ws, size_t ws_bytes, cudaStream_t st,
                   int budget_sms, bool pdl) {
   const int sms = budget_sms > 0 && budget_sms < c->num_sms ? budget_sms : c->num_sms;
-  if (c->p.type_k != c->p.type_v) return KVQ_E_UNSUPPORTED;
+  // K and V of different types: a Q.K kernel of the K type writes the scores, a P.V kernel of
+  // the V type reads them (not overlapped with a preceding append)
+  const bool mixed = c->p.type_k != c->p.type_v;
+  if (mixed && (c->fam_k == FAM_BF16 || c->fam_v == FAM_BF16)) return KVQ_E_UNSUPPORTED;
+  if (mixed) pdl = false;
   (void)ws_bytes;
   const LayerView L = layer_view(c, layer);
   const int hkv = c->p.n_kv_heads, G = n_q_heads / hkv;
@@ -1317,6 +1407,8 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
     A.q = q;
     A.out = out;
     A.ws = static_cast<float *>(ws);
+    A.scores = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode_partials_bytes(c, (int)seqs.size(), n_q_heads));
+    A.qcap = decode_score_cap(c);
     A.tickets = reinterpret_cast<uint32_t *>(c->base + c->off_tickets);
     // split plan (min-max greedy): every (sequence, part) with tokens starts with one split
     // per KV head; then, while a whole column of hkv CTAs still fits in one wave, the part
@@ -1371,7 +1463,14 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
     A.ncta = cta;
     // q / out rows are indexed by DecodeSeq::row; the workspace slots restart per launch
     // overlap only a decode of one launch: a second launch would follow the first, not the producer
-    if (dispatch(c->fam_k, c->bits_k, L, A, st, pdl && seqs.size() <= (size_t)MAXS) != cudaSuccess)
+    if (mixed) {
+      if (dispatch(c->fam_k, c->bits_k, M_SCORES, L, A, st, false) != cudaSuccess ||
+          dispatch(c->fam_v, c->bits_v, M_PVEXT, L, A, st, false) != cudaSuccess)
+        return KVQ_E_CUDA;
+      note_launches(2);
+      continue;
+    }
+    if (dispatch(c->fam_k, c->bits_k, M_FUSED, L, A, st, pdl && seqs.size() <= (size_t)MAXS) != cudaSuccess)
       return KVQ_E_CUDA;
     note_launches(1);
   }

@@ -84,16 +84,22 @@ typedef struct kvq_params {
   int32_t n_kv_heads;     /* >= 1 */
   int32_t head_dim;       /* must be 128 */
   int64_t max_ctx;        /* tokens per sequence, >= 1 */
-  int32_t type_k, type_v; /* kvq_type; BF16 must be used for both or neither */
+  int32_t type_k, type_v; /* kvq_type, chosen independently; BF16 must be used for both
+                           * or neither (KVQ_E_UNSUPPORTED) */
   int32_t tail;           /* newest tokens kept in BF16, >= 0 */
   int32_t group;          /* kvarn group length, must be 256 */
   int32_t sinkhorn_iters; /* Sinkhorn iterations, 1..64 (8 by default) */
   int32_t page_tokens;    /* tokens per page, must be 256 */
+  int32_t var_norm;       /* 0 or 1: KVarN variance normalization on the qN_0 types, the
+                           * pages' --cache-var-norm switch ("KVarN" section of the BeeLLama.cpp
+                           * v0.4.0 page): qN_0 with it is stored as kvarnN (rotation, Sinkhorn,
+                           * then the same symmetric quantizer); kvarn types are unchanged; BF16
+                           * and the qN_1 types with it are KVQ_E_UNSUPPORTED */
 } kvq_params;
 
 typedef struct kvq_cache kvq_cache;
 
-/* Default parameters (head_dim 128, group 256, page 256, 8 iterations, tail 1024). */
+/* Default parameters (head_dim 128, group 256, page 256, 8 iterations, tail 1024, no var_norm). */
 void kvq_default_params(kvq_params *p);
 
 /* Bytes of device memory a cache with these parameters needs (host-only arithmetic).
@@ -126,7 +132,9 @@ void kvq_cache_destroy(kvq_cache *c);
 int kvq_append(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,
                const int32_t *n_new, const void *k_bf16, const void *v_bf16, kvq_stream_t stream);
 
-/* Workspace bytes kvq_decode_attn needs for n_seqs sequences and n_q_heads heads. */
+/* Workspace bytes kvq_decode_attn needs for n_seqs sequences and n_q_heads heads: the
+ * split-K partials, and, when type_k != type_v, also the Q.K scores of the quantized prefix
+ * (4 bytes x min(n_seqs, 64) x n_q_heads x max_ctx rounded up to 32). */
 int kvq_workspace_bytes(const kvq_cache *c, int32_t n_seqs, int32_t n_q_heads, size_t *bytes);
 
 /* Decode attention of one query token per sequence over [quantized prefix | BF16 tail].
@@ -134,6 +142,10 @@ int kvq_workspace_bytes(const kvq_cache *c, int32_t n_seqs, int32_t n_q_heads, s
  * softmax_scale <= 0 selects 1/sqrt(128).  n_q_heads must be a multiple of n_kv_heads
  * with n_q_heads / n_kv_heads <= 8.  Split-K over the context; the last block of each
  * (sequence, KV head) merges the splits.  workspace: device, >= kvq_workspace_bytes.
+ * K and V of one type run as one kernel; different types (the pages' separate
+ * --cache-type-k / --cache-type-v) as two over the same split plan: Q.K of the K type
+ * writes the scores of the quantized prefix to the workspace, then softmax and P.V of
+ * the V type, the BF16 tail and the merge read them.
  * A sequence with no tokens gives zeros.  Decodes of one cache must not overlap on the
  * GPU (they share per-cache merge counters). */
 int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,
@@ -164,7 +176,8 @@ int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_token
  * kernel: its warps start on pages the append does not touch while the append runs, and
  * wait for it (griddepcontrol.wait) only before the pages and ring rows it rewrites.  When
  * that kernel is a small spill (a one-token step), the decode's split plan leaves the
- * spill's SMs out.  Requirements beyond the two calls': q must be complete before this call
+ * spill's SMs out.  With type_k != type_v the decode follows the append in plain stream
+ * order instead.  Requirements beyond the two calls': q must be complete before this call
  * is issued (it is read while the append runs), and nothing else may be enqueued on `stream`
  * in between (there is nothing in between: this is one call).  Errors: those of the two
  * calls, all checked before anything is launched. */

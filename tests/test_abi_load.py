@@ -50,3 +50,23 @@ def test_host_validation_and_sizes():
         kvq.kvq_cache_create(p, 8, nb)  # misaligned pointer is rejected before any device call
     assert e.value.code == kvq.KVQ_E_ALIGN
     assert kvq.kvq_strerror(kvq.KVQ_E_CAPACITY).startswith("sequence capacity")
+
+
+def test_var_norm_resolves_to_the_kvarn_type():
+    """The pages' --cache-var-norm switch: qN_0 with KVarN normalization is kvarnN (same
+    rotation, balancing and symmetric quantizer); qN_1 and BF16 have no such form."""
+    from bit_kv_cache_17_b200 import kvq
+
+    for b in (2, 3, 4, 5, 6, 8):
+        a = kvq.kvq_cache_bytes(kvq.kvq_default_params(type_k=f"q{b}_0", type_v=f"q{b}_0", var_norm=1))
+        r = kvq.kvq_cache_bytes(kvq.kvq_default_params(type_k=f"kvarn{b}", type_v=f"kvarn{b}"))
+        assert a == r
+    assert kvq.kvq_cache_bytes(kvq.kvq_default_params(type_k="kvarn4", type_v="kvarn4", var_norm=1)) == \
+        kvq.kvq_cache_bytes(kvq.kvq_default_params(type_k="kvarn4", type_v="kvarn4"))
+    for t in ("q4_1", "bf16"):
+        with pytest.raises(kvq.KVQError) as e:
+            kvq.kvq_cache_bytes(kvq.kvq_default_params(type_k=t, type_v=t, var_norm=1))
+        assert e.value.code == kvq.KVQ_E_UNSUPPORTED
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.kvq_cache_bytes(kvq.kvq_default_params(var_norm=2))
+    assert e.value.code == kvq.KVQ_E_INVAL
