@@ -15,6 +15,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <cstddef>
 
 #include "kvq_codes.cuh"
 #include "kvq_internal.h"
@@ -426,12 +427,13 @@ __device__ __forceinline__ void copy_chunk(const LayerView &L, int seq, int head
 
 // Per-warp scale tables of one chunk, built with one token per lane.
 template <int FAM>
-struct ChunkTabs {
+struct alignas(16) ChunkTabs {
   static constexpr int NM = FAM == FAM_ASYM ? CH : 1;
-  float k[CH / 2][4][2];  // K: d * t (kvarn) or d, per token pair, block, token (0 past the end)
-  float v[4][CH];         // V: t * d * QFIX / max over the chunk (per block) -> weights in fixed point
-  float km[NM][4];        // qb_1 K: m + d * 2^(b-1)
-  float vm[NM][4];        // qb_1 V: m + d * 2^(b-1)
+  // (read with 8- and 16-byte vector loads: each member starts on 16 bytes)
+  alignas(16) float k[CH / 2][4][2];  // K: d * t (kvarn) or d, per token pair, block, token (0 past the end)
+  alignas(16) float v[4][CH];  // V: t * d * QFIX / max over the chunk (per block) -> weights in fixed point
+  alignas(16) float km[NM][4];  // qb_1 K: m + d * 2^(b-1)
+  alignas(16) float vm[NM][4];  // qb_1 V: m + d * 2^(b-1)
 };
 
 
@@ -1034,20 +1036,37 @@ __device__ __forceinline__ void warp_wht(float (&v)[4], int lane) {
 
 // Shared memory of the kernel (dynamic): fixed part + per-warp stage area (also used for the
 // warps' accumulators once the chunks are done).
+// What the end of the kernel (CTA combine, ticket, merge) needs of the launch arguments, kept
+// in shared memory from the start: the entry table is indexed at run time, and reading it again
+// after the main loop costs constant-cache misses of about a microsecond each.
+struct CtaMeta {
+  float *rec;        // this (entry, KV head)'s split records: [split][G][PSTRIDE]
+  float *out;        // this (entry, KV head)'s output rows: [G][D]
+  uint32_t *ticket;  // its merge ticket
+  int G, sp, nspl, nsq, rotv;
+};
+
 template <int NW, int FAM>
 struct SmemFixed {
-  float qraw[MAX_G][D];
-  float qrot[MAX_G][D];
+  CtaMeta meta;
+  // q, q' and the merge sums are read and written with 16-byte vector accesses
+  alignas(16) float qraw[MAX_G][D];
+  alignas(16) float qrot[MAX_G][D];
   float mw[NW][MAX_G], lw[NW][MAX_G];
   float fw[MAXSPL][MAX_G];   // weight of each warp (CTA combine) / split (merge)
   float fm[MAXSPL][MAX_G];   // merge: m and l of the splits whose records are not staged
   float fl[MAXSPL][MAX_G];
-  float red[MAX_G][D];       // merge: sum over the tail splits (original basis)
+  alignas(16) float red[MAX_G][D];  // merge: sum over the tail splits (original basis)
   float Ls[MAX_G];
   float Mc[MAX_G], Lc[MAX_G];  // this CTA's combined m and l per head
   ChunkTabs<FAM> tabs[NW];
   int is_last;
 };
+using SmemFixedA12 = SmemFixed<12, FAM_ASYM>;
+using SmemFixedK8 = SmemFixed<8, FAM_KVARN>;
+static_assert(offsetof(SmemFixedA12, qrot) % 16 == 0 && offsetof(SmemFixedK8, tabs) % 16 == 0 &&
+                  offsetof(SmemFixedK8, red) % 16 == 0,
+              "vector-accessed shared arrays start on 16 bytes");
 
 template <int FAM, int BITS>
 __host__ __device__ constexpr int warp_area() {
@@ -1132,20 +1151,42 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   bool waited = false;
   PageCursor pc;
   const ScoreRow sr{A.scores + (int64_t)(si * A.hkv + head) * G * A.qcap, A.qcap};
+  // the query rows of this KV head are loaded first, so that they do not queue behind the
+  // prefetched chunks of every CTA
+  constexpr int QPER = (MAX_G * D + DT - 1) / DT;
+  float qv[QPER];
+#pragma unroll
+  for (int u = 0; u < QPER; ++u) {
+    const int idx = tid + u * DT, g = idx / D, j = idx % D;
+    qv[u] = (idx < MAX_G * D && g < G) ? __ldg(&A.q[((int64_t)s.row * A.hkv * G + head * G + g) * D + j]) : 0.f;
+  }
   if constexpr (FAM != FAM_BF16) {
     if (!tail)
       warp_quant_prefetch<FAM, BITS, MODE>(L, s.seq, head, a, (int)c0, (int)c1, cdirty, waited,
                                            warp_mem + (size_t)warp * WA, lane, pc,
                                            page_area<FAM, BITS>(warp_mem + (size_t)warp * WA), sr, G);
   }
-  // query rows of this KV head, pre-scaled by softmax_scale * log2(e); heads >= G are 0
-  for (int idx = tid; idx < MAX_G * D; idx += DT) {
-    const int g = idx / D, j = idx % D;
-    F.qraw[g][j] = g < G ? A.q[((int64_t)s.row * A.hkv * G + head * G + g) * D + j] * A.qscale : 0.f;
+  // query rows, pre-scaled by softmax_scale * log2(e); heads >= G are 0
+#pragma unroll
+  for (int u = 0; u < QPER; ++u) {
+    const int idx = tid + u * DT;
+    if (idx < MAX_G * D) F.qraw[idx / D][idx % D] = qv[u] * A.qscale;
   }
   for (int idx = tid; idx < NW * MAX_G; idx += DT) {
     F.mw[idx / MAX_G][idx % MAX_G] = -INFINITY;
     F.lw[idx / MAX_G][idx % MAX_G] = 0.f;
+  }
+  if (tid == 0) {
+    CtaMeta m;
+    m.rec = A.ws + (int64_t)(s.part0 + head * nspl) * G * PSTRIDE;
+    m.out = A.out + ((int64_t)s.row * A.hkv * G + head * G) * D;
+    m.ticket = &A.tickets[si * A.hkv + head];
+    m.G = G;
+    m.sp = sp;
+    m.nspl = nspl;
+    m.nsq = s.nsq;
+    m.rotv = A.rotv;
+    F.meta = m;
   }
   __syncthreads();
   // BF16 rows (the tail splits, or a whole BF16 cache) take the raw q as bf16 MMA fragments,
@@ -1186,9 +1227,11 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   }
   __syncthreads();
 
+  const CtaMeta mt = F.meta;
+  {
+    const int G = mt.G;  // (shadows the launch argument: from here on only shared memory)
   // combine the warps of this CTA into its partial (m, l, acc) per query head: warp g
   // reduces head g over the warps, one lane per warp
-  const int slot0 = s.part0 + head * nspl;
   if (warp < G) {
     const float mw = lane < NW ? F.mw[lane][warp] : -INFINITY;
     const float M = warp_max(mw);
@@ -1207,7 +1250,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
 #pragma unroll 4
     for (int w = 0; w < NW; ++w)
       av = fmaf(F.fw[w][g], reinterpret_cast<const float *>(warp_mem + (size_t)w * WA)[g * D + c], av);
-    float *dst = A.ws + ((int64_t)(slot0 + sp) * G + g) * PSTRIDE;
+    float *dst = mt.rec + (int64_t)(mt.sp * G + g) * PSTRIDE;
     dst[PACC + c] = av;
     if (c == 0) {
       dst[0] = F.Mc[g];
@@ -1215,21 +1258,25 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
     }
   }
 
-  // the last CTA of this (sequence, KV head) merges all splits (atomic ticket; no waiting)
-  __threadfence();
+  // the last CTA of this (sequence, KV head) merges all splits (atomic ticket; no waiting).
+  // The barrier orders the CTA's record stores before thread 0's fence and ticket (release);
+  // in the last CTA, thread 0's second fence and the barrier order the other records before
+  // every thread's reads (acquire).
   __syncthreads();
   if (tid == 0) {
-    const unsigned prev = atomicAdd(&A.tickets[si * A.hkv + head], 1u);
-    F.is_last = prev == (unsigned)(nspl - 1);
+    __threadfence();
+    const unsigned prev = atomicAdd(mt.ticket, 1u);
+    F.is_last = prev == (unsigned)(mt.nspl - 1);
+    if (F.is_last) __threadfence();
   }
   __syncthreads();
   if (!F.is_last) return;
-  __threadfence();
 
   // The partial records (nspl * G of them, contiguous) are staged in shared memory by cp.async,
   // as many whole splits per batch as the warp areas hold; the m and l of the splits beyond
   // the first batch are read directly, so that the weights are known before any sum.
-  const float *part = A.ws + (int64_t)slot0 * G * PSTRIDE;
+  const int nspl = mt.nspl;
+  const float *part = mt.rec;
   float *stage = reinterpret_cast<float *>(warp_mem);
   constexpr int CAP = (NW * WA) / (PSTRIDE * 4);  // records that fit
   const int kper = CAP / G;                       // whole splits per batch (>= 1)
@@ -1275,7 +1322,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
       float srot = kb0 ? F.qraw[g][ch] : 0.f, spl = kb0 ? F.red[g][ch] : 0.f;
       for (int k = kb0; k < kb1; ++k) {
         const float v = stage[((k - kb0) * G + g) * PSTRIDE + PACC + ch];
-        if (k < s.nsq)
+        if (k < mt.nsq)
           srot = fmaf(F.fw[k][g], v, srot);
         else
           spl = fmaf(F.fw[k][g], v, spl);
@@ -1299,7 +1346,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
     float v[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) v[e] = F.qraw[g][4 * lane + e];
-    if (A.rotv) {
+    if (mt.rotv) {
       warp_wht(v, lane);
 #pragma unroll
       for (int e = 0; e < 4; ++e) v[e] *= kKappa();
@@ -1311,9 +1358,10 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
     o.y = (v[1] + F.red[g][4 * lane + 1]) * inv;
     o.z = (v[2] + F.red[g][4 * lane + 2]) * inv;
     o.w = (v[3] + F.red[g][4 * lane + 3]) * inv;
-    *reinterpret_cast<float4 *>(A.out + ((int64_t)s.row * A.hkv * G + head * G + g) * D + 4 * lane) = o;
+    *reinterpret_cast<float4 *>(mt.out + (int64_t)g * D + 4 * lane) = o;
   }
-  if (tid == 0) A.tickets[si * A.hkv + head] = 0u;
+  if (tid == 0) *mt.ticket = 0u;
+  }
 }
 
 template <int FAM, int BITS, int MODE>
