@@ -60,6 +60,7 @@ int check_params(const kvq_params *p) {
     return KVQ_E_INVAL;
   if (p->head_dim != D || p->group != GROUP || p->page_tokens != GROUP) return KVQ_E_UNSUPPORTED;
   if (p->sinkhorn_iters < 1 || p->sinkhorn_iters > 64) return KVQ_E_INVAL;
+  if (p->tail_f16 != 0 && p->tail_f16 != 1) return KVQ_E_INVAL;
   TypeInfo tk = type_info(p->type_k), tv = type_info(p->type_v);
   if (tk.fam < 0 || tv.fam < 0) return KVQ_E_UNSUPPORTED;
   if ((tk.fam == FAM_BF16) != (tv.fam == FAM_BF16)) return KVQ_E_UNSUPPORTED;
@@ -118,6 +119,7 @@ LayerView layer_view(const kvq_cache *c, int layer) {
   L.sub_v = c->lv.bytes;
   L.type_k = c->p.type_k;
   L.type_v = c->p.type_v;
+  L.tail_f16 = c->p.tail_f16;
   return L;
 }
 }  // namespace kvq
@@ -418,9 +420,10 @@ const char *kvq_describe(kvq_cache *c) {
   if (!c) return "";
   char buf[512];
   snprintf(buf, sizeof buf,
-           "kvq cache: K %s, V %s, tail %d (BF16), %d layers x %d seqs x %d KV heads x %d, max_ctx %lld, "
+           "kvq cache: K %s, V %s, tail %d (%s), %d layers x %d seqs x %d KV heads x %d, max_ctx %lld, "
            "sinkhorn_iters %d, %zu bytes (pages %zu/layer, ring %zu/layer)",
-           type_name(c->p.type_k), type_name(c->p.type_v), c->p.tail, c->p.n_layers, c->p.n_seqs,
+           type_name(c->p.type_k), type_name(c->p.type_v), c->p.tail, c->p.tail_f16 ? "F16" : "BF16", c->p.n_layers,
+           c->p.n_seqs,
            c->p.n_kv_heads, c->p.head_dim, (long long)c->p.max_ctx, c->p.sinkhorn_iters, c->total,
            c->layer_pages_bytes, c->layer_ring_bytes);
   c->desc = buf;

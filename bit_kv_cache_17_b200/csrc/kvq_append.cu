@@ -57,14 +57,21 @@ __device__ __forceinline__ const __nv_bfloat16 *src_row(const LayerView &L, cons
   return in + ((s.in_off + (p - s.n0)) * L.hkv + head) * D;
 }
 
-__device__ __forceinline__ void load4(const __nv_bfloat16 *row, int lane, float (&x)[4]) {
-  uint2 raw = *reinterpret_cast<const uint2 *>(row + 4 * lane);
-  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
-  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
-  x[0] = __low2float(a);
-  x[1] = __high2float(a);
-  x[2] = __low2float(b);
-  x[3] = __high2float(b);
+// channels 4 lane .. 4 lane + 3 of token p as the quantizer sees them: a ring row as stored,
+// an input row rounded to the tail's format
+__device__ __forceinline__ void load4(const LayerView &L, const SeqWork &s, int head, int which, int64_t p,
+                                      const __nv_bfloat16 *in, int lane, float (&x)[4]) {
+  const bool ring = p < s.n0;
+  const uint2 raw = *reinterpret_cast<const uint2 *>(src_row(L, s, head, which, p, in) + 4 * lane);
+  const float2 a = ring2f(raw.x, ring ? L.tail_f16 : 0), b = ring2f(raw.y, ring ? L.tail_f16 : 0);
+  x[0] = a.x;
+  x[1] = a.y;
+  x[2] = b.x;
+  x[3] = b.y;
+  if (!ring && L.tail_f16) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = tail_round(x[e], 1);
+  }
 }
 
 // ---- packing -------------------------------------------------------------------------
@@ -216,7 +223,7 @@ __global__ void __launch_bounds__(256) k_spill_qb(LayerView L, Work W, const __n
   const SubLayout lay = sub_layout(FAM, BITS);
   uint8_t *sub = subpage_ptr(L, s.seq, p / GROUP, head, WHICH);
   float x[4];
-  load4(src_row(L, s, head, WHICH, p, in), lane, x);
+  load4(L, s, head, WHICH, p, in, lane, x);
   const int tip = (int)(p % GROUP);
   if constexpr (FAM == FAM_SYM)
     quant_sym<BITS, WHICH>(x, sub, lay, tip, lane);
@@ -442,7 +449,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
   if (g0 + GROUP >= Q1) {
     for (int64_t p = s.tw + tid / 16; p < s.n1; p += KV_THREADS / 16) {
       const uint4 *src = reinterpret_cast<const uint4 *>(in + ((s.in_off + (p - s.n0)) * L.hkv + head) * D);
-      reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, which, p))[tid & 15] = src[tid & 15];
+      reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, which, p))[tid & 15] = bf16x8_to_ring(src[tid & 15], L.tail_f16);
     }
   }
 
@@ -454,6 +461,9 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     const int row = tid >> 1, h = tid & 1;
     if (row < ng) {
       const uint4 *src = reinterpret_cast<const uint4 *>(src_row(L, s, head, which, g0 + row, in));
+      // a ring row as stored; an input row rounded to the tail's format (F16 tails)
+      const bool ring = g0 + row < s.n0;
+      const int f16r = ring ? L.tail_f16 : 0, rnd = ring ? 0 : L.tail_f16;
       float r[D / 2];  // r[i] = channel 2i + h
 #pragma unroll
       for (int j8 = 0; j8 < D / 8; ++j8) {
@@ -461,7 +471,12 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+          float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+          if (f16r | rnd) {
+            const float2 xf = ring2f(w[u], f16r);
+            x0 = tail_round(xf.x, rnd);
+            x1 = tail_round(xf.y, rnd);
+          }
           r[4 * j8 + u] = h ? __fsub_rn(x0, x1) : __fadd_rn(x0, x1);
         }
       }
@@ -648,7 +663,7 @@ __global__ void __launch_bounds__(256) k_tail_write(LayerView L, Work W, const _
   const int64_t p = s.a + local / L.hkv;
   const uint4 *src = reinterpret_cast<const uint4 *>(in + ((s.in_off + (p - s.n0)) * L.hkv + head) * D);
   uint4 *dst = reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, which, p));
-  dst[part] = src[part];
+  dst[part] = bf16x8_to_ring(src[part], L.tail_f16);
 }
 
 // ---- dispatch ----------------------------------------------------------------------------

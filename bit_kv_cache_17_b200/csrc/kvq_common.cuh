@@ -117,6 +117,7 @@ struct LayerView {
   int32_t hkv;
   int32_t sub_k, sub_v;  // sub-page bytes of K and V
   int32_t type_k, type_v;
+  int32_t tail_f16;      // the ring holds F16 rows (else BF16)
 };
 
 __device__ __forceinline__ uint8_t *subpage_ptr(const LayerView &L, int seq, int64_t page, int head,
@@ -125,6 +126,32 @@ __device__ __forceinline__ uint8_t *subpage_ptr(const LayerView &L, int seq, int
   return L.pages + phys * L.page_bytes + (int64_t)head * (L.sub_k + L.sub_v) + (which ? L.sub_k : 0);
 }
 
+// ---- the tail's 16-bit format ------------------------------------------------------------
+// The ring holds BF16 rows, or F16 rows for a cache with an F16 tail.  An F16 tail stores
+// fp16(x) of each BF16 input x (round to nearest even, overflow to inf), and the quantizer
+// reads that same value whether the token comes from the ring or straight from the input.
+// (Every fp16 rounding of a BF16 value is again a BF16 value, so such a stream is the BF16
+// stream of the rounded inputs.)
+__device__ __forceinline__ float tail_round(float x, int f16) { return f16 ? __half2float(__float2half_rn(x)) : x; }
+
+// two 16-bit ring elements (one 32-bit word, element 0 low) as floats
+__device__ __forceinline__ float2 ring2f(uint32_t w, int f16) {
+  if (f16) return __half22float2(*reinterpret_cast<const __half2 *>(&w));
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// two BF16 input elements (one word) as the ring stores them
+__device__ __forceinline__ uint32_t bf16w_to_ring(uint32_t w, int f16) {
+  if (!f16) return w;
+  const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+__device__ __forceinline__ uint4 bf16x8_to_ring(uint4 v, int f16) {
+  if (!f16) return v;
+  return make_uint4(bf16w_to_ring(v.x, 1), bf16w_to_ring(v.y, 1), bf16w_to_ring(v.z, 1), bf16w_to_ring(v.w, 1));
+}
+
+// ring row of a token (16-bit elements, BF16 or F16 by the cache's tail format)
 __device__ __forceinline__ __nv_bfloat16 *ring_row(const LayerView &L, int seq, int head, int which,
                                                    int64_t token) {
   int64_t slot = token % L.ring_cap;

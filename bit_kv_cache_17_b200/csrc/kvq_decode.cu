@@ -820,9 +820,11 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
   }
 }
 
-// ---- exact BF16 rows (the tail, or a whole BF16 cache) on the tensor cores ---------------
+// ---- exact 16-bit rows (the tail, or a whole BF16 cache) on the tensor cores -------------
 //
-// mma.sync m16n8k16, bf16 x bf16 -> fp32.  Q.K: A = the queries, rows 0..7 the bf16 high
+// mma.sync m16n8k16, bf16 x bf16 -> fp32 (f16 x f16 for a cache with an F16 tail; the
+// description below says bf16 for both).  F16 high part + remainder carry about 22 bits of
+// the query; values below the f16 normal range keep an absolute precision of 2^-25.  Q.K: A = the queries, rows 0..7 the bf16 high
 // part of head g and rows 8..15 the bf16 remainder q - hi (together about 16 significant
 // bits); B = K^T, 8 tokens per n-tile, read straight from the BF16 ring with 16-byte loads:
 // within a 32-channel step s the k order is permuted so that lane (g, tq) supplies channels
@@ -833,11 +835,18 @@ __device__ __forceinline__ void warp_quant(const LayerView &L, int seq, int head
 // n-tile (j, e) is channel 8 (8 j + n) + e, so a lane's loads are whole 16-byte pieces.  The
 // P.V accumulators stay in fp32 across the whole split (no per-chunk epilogue).
 
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+template <bool F16>
+__device__ __forceinline__ void mma_16(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
+  if constexpr (F16)
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+  else
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
 }
 
 // (lo, hi) -> bf16x2 with lo in the low half, each rounded to nearest even
@@ -855,15 +864,38 @@ __device__ __forceinline__ void bf16_split(float x0, float x1, uint32_t &hi, uin
   lo = bf16x2_rn(x0 - bf_lo(hi), x1 - bf_hi(hi));
 }
 
+// the same split in f16
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<const uint32_t *>(&h); }
+__device__ __forceinline__ void f16_split(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  hi = h2u(h);
+  lo = h2u(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
+}
+
+template <bool F16>
+__device__ __forceinline__ void split16(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  if constexpr (F16)
+    f16_split(x0, x1, hi, lo);
+  else
+    bf16_split(x0, x1, hi, lo);
+}
+
 // Query fragments of the BF16 path for one KV head (all warps of the CTA share them):
 // qfb[ks * 32 + lane] = (a0, a1, a2, a3) of k-step ks = 2 s + h.
-__device__ __forceinline__ void build_qfrag_bf16(uint4 *qfb, const float (*qraw)[D], int tid, int nthreads) {
+__device__ __forceinline__ void build_qfrag_bf16(uint4 *qfb, const float (*qraw)[D], int tid, int nthreads,
+                                                 int f16) {
   for (int t = tid; t < 8 * 32; t += nthreads) {
     const int ks = t >> 5, l = t & 31, g = l >> 2, tq = l & 3;
     const int c = 32 * (ks >> 1) + 8 * tq + 4 * (ks & 1);
     uint4 f;
-    bf16_split(qraw[g][c], qraw[g][c + 1], f.x, f.y);
-    bf16_split(qraw[g][c + 2], qraw[g][c + 3], f.z, f.w);
+    if (f16) {
+      f16_split(qraw[g][c], qraw[g][c + 1], f.x, f.y);
+      f16_split(qraw[g][c + 2], qraw[g][c + 3], f.z, f.w);
+    } else {
+      bf16_split(qraw[g][c], qraw[g][c + 1], f.x, f.y);
+      bf16_split(qraw[g][c + 2], qraw[g][c + 3], f.z, f.w);
+    }
     qfb[t] = f;
   }
 }
@@ -873,7 +905,7 @@ __device__ __forceinline__ void build_qfrag_bf16(uint4 *qfb, const float (*qraw)
 // V loads are replaced by zeros and their scores by -inf.  NJ = 2 accumulates all 128
 // channels in one pass over the tokens; NJ = 1 takes two passes of 64 channels (columns
 // n-tile j = pass), recomputing the identical scores, with half the accumulator registers.
-template <int NJ>
+template <int NJ, bool F16>
 __device__ __forceinline__ void warp_bf16_tc(const LayerView &L, int seq, int head, int64_t a, int64_t b, int64_t c0,
                                              int64_t c1, int64_t cdirty, const uint4 *qfb, float *mw, float *lw,
                                              float *accw) {
@@ -918,8 +950,8 @@ __device__ __forceinline__ void warp_bf16_tc(const LayerView &L, int seq, int he
         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int s2 = 0; s2 < 4; ++s2) {
-          mma_bf16(d, qfb[(2 * s2) * 32 + lane], kr[s2].x, kr[s2].y);
-          mma_bf16(d, qfb[(2 * s2 + 1) * 32 + lane], kr[s2].z, kr[s2].w);
+          mma_16<F16>(d, qfb[(2 * s2) * 32 + lane], kr[s2].x, kr[s2].y);
+          mma_16<F16>(d, qfb[(2 * s2 + 1) * 32 + lane], kr[s2].z, kr[s2].w);
         }
         sc[2 * nt] = 8 * nt + 2 * tq < nvalid ? d[0] + d[2] : -INFINITY;
         sc[2 * nt + 1] = 8 * nt + 2 * tq + 1 < nvalid ? d[1] + d[3] : -INFINITY;
@@ -952,8 +984,8 @@ __device__ __forceinline__ void warp_bf16_tc(const LayerView &L, int seq, int he
 #pragma unroll
       for (int kt = 0; kt < 2; ++kt) {
         uint4 pa;  // rows g / g+8: weights of tokens 16 kt + 2tq + (0, 1) and 16 kt + 8 + 2tq + (0, 1)
-        bf16_split(p[4 * kt], p[4 * kt + 1], pa.x, pa.y);
-        bf16_split(p[4 * kt + 2], p[4 * kt + 3], pa.z, pa.w);
+        split16<F16>(p[4 * kt], p[4 * kt + 1], pa.x, pa.y);
+        split16<F16>(p[4 * kt + 2], p[4 * kt + 3], pa.z, pa.w);
         int sl[4];
         bool vl[4];
 #pragma unroll
@@ -978,7 +1010,7 @@ __device__ __forceinline__ void warp_bf16_tc(const LayerView &L, int seq, int he
             const uint32_t w1 = w == 0 ? rv[1].x : (w == 1 ? rv[1].y : (w == 2 ? rv[1].z : rv[1].w));
             const uint32_t w2 = w == 0 ? rv[2].x : (w == 1 ? rv[2].y : (w == 2 ? rv[2].z : rv[2].w));
             const uint32_t w3 = w == 0 ? rv[3].x : (w == 1 ? rv[3].y : (w == 2 ? rv[3].z : rv[3].w));
-            mma_bf16(acc[j][e], pa, __byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel));
+            mma_16<F16>(acc[j][e], pa, __byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel));
           }
         }
       }
@@ -1195,7 +1227,7 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   uint4 *qfb = reinterpret_cast<uint4 *>(&F.qrot[0][0]);
   static_assert(sizeof(F.qrot) >= 8 * 32 * sizeof(uint4), "q' area holds the BF16 query fragments");
   if (bf16_rows) {
-    build_qfrag_bf16(qfb, F.qraw, tid, DT);
+    build_qfrag_bf16(qfb, F.qraw, tid, DT, L.tail_f16);
   } else if (MODE == M_PVEXT) {
     // the scores are given: no query on the quantized splits
   } else if (A.rotk) {
@@ -1223,7 +1255,11 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
     if constexpr (MODE == M_SCORES) return;  // every CTA of this kernel is a quantized split
   } else {
     // quantized kernels keep their tail warps light on registers: two channel passes
-    warp_bf16_tc<FAM == FAM_BF16 ? 2 : 1>(L, s.seq, head, a, b, c0, c1, cdirty, qfb, F.mw[warp], F.lw[warp], accw);
+    constexpr int NJ = FAM == FAM_BF16 ? 2 : 1;
+    if (L.tail_f16)
+      warp_bf16_tc<NJ, true>(L, s.seq, head, a, b, c0, c1, cdirty, qfb, F.mw[warp], F.lw[warp], accw);
+    else
+      warp_bf16_tc<NJ, false>(L, s.seq, head, a, b, c0, c1, cdirty, qfb, F.mw[warp], F.lw[warp], accw);
   }
   __syncthreads();
 

@@ -26,9 +26,12 @@ __global__ void __launch_bounds__(256)
   const int head = (int)(item % L.hkv);
   float v[4];
   if (FAM == FAM_BF16 || p >= Q) {
-    const __nv_bfloat16 *row = ring_row(L, seq, head, which, p);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] = __bfloat162float(row[4 * lane + e]);
+    const uint2 raw = *reinterpret_cast<const uint2 *>(ring_row(L, seq, head, which, p) + 4 * lane);
+    const float2 a = ring2f(raw.x, L.tail_f16), b = ring2f(raw.y, L.tail_f16);
+    v[0] = a.x;
+    v[1] = a.y;
+    v[2] = b.x;
+    v[3] = b.y;
   } else {
     if constexpr (FAM != FAM_BF16) {
       const SubLayout lay = sub_layout(FAM, BITS);

@@ -29,7 +29,7 @@ class kvq_params(C.Structure):
         ("n_layers", C.c_int32), ("n_seqs", C.c_int32), ("n_kv_heads", C.c_int32),
         ("head_dim", C.c_int32), ("max_ctx", C.c_int64), ("type_k", C.c_int32),
         ("type_v", C.c_int32), ("tail", C.c_int32), ("group", C.c_int32),
-        ("sinkhorn_iters", C.c_int32), ("page_tokens", C.c_int32), ("var_norm", C.c_int32),
+        ("sinkhorn_iters", C.c_int32), ("page_tokens", C.c_int32), ("var_norm", C.c_int32), ("tail_f16", C.c_int32),
     ]
 
 

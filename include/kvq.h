@@ -95,11 +95,18 @@ typedef struct kvq_params {
                            * v0.4.0 page): qN_0 with it is stored as kvarnN (rotation, Sinkhorn,
                            * then the same symmetric quantizer); kvarn types are unchanged; BF16
                            * and the qN_1 types with it are KVQ_E_UNSUPPORTED */
+  int32_t tail_f16;       /* 0: the 16-bit tail (and a BF16 cache) holds BF16 rows; 1: F16
+                           * rows (the pages' "last N tokens in BF16/F16", "KV Cache
+                           * Precision Tail").  An F16 tail stores fp16(x) of each BF16
+                           * input x (round to nearest even; beyond +-65504 it overflows to
+                           * inf, as any F16 cache), and tokens are quantized from that same
+                           * value.  Other values: KVQ_E_INVAL */
 } kvq_params;
 
 typedef struct kvq_cache kvq_cache;
 
-/* Default parameters (head_dim 128, group 256, page 256, 8 iterations, tail 1024, no var_norm). */
+/* Default parameters (head_dim 128, group 256, page 256, 8 iterations, tail 1024, no var_norm,
+ * BF16 tail). */
 void kvq_default_params(kvq_params *p);
 
 /* Bytes of device memory a cache with these parameters needs (host-only arithmetic).

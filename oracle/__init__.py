@@ -114,6 +114,23 @@ def f16_to_f32(h):
     return y
 
 
+def f16_tail_bits(x_bf16):
+    """The F16 tail's stored value of each BF16 input ("KV Cache Precision Tail": the newest
+    tokens stay 16-bit, BF16 or F16): fp16 round to nearest even, overflow to inf."""
+    return f32_to_f16(bf16_to_f32(x_bf16))
+
+
+def f16_tail_rows(x_bf16):
+    """The values a stream with an F16 tail holds and quantizes, as BF16 bits.  Every fp16
+    rounding of a BF16 value is again a BF16 value (checked here), so that stream is the
+    BF16-tail stream of these rows."""
+    y = f16_to_f32(f16_tail_bits(x_bf16))
+    b = f32_to_bf16(y)
+    back = bf16_to_f32(b)
+    assert np.array_equal(back[~np.isnan(y)], y[~np.isnan(y)])
+    return b
+
+
 def wht128(v):
     v = _c(v, np.float32).copy()
     assert v.shape[-1] == D

@@ -16,11 +16,11 @@ def torch():
     return t
 
 
-def make_cache(type_k, hkv, max_ctx, tail, n_seqs=1, n_layers=1, type_v=None, iters=8):
+def make_cache(type_k, hkv, max_ctx, tail, n_seqs=1, n_layers=1, type_v=None, iters=8, tail_f16=0):
     from bit_kv_cache_17_b200.kvq import KVCache
 
     return KVCache(n_layers=n_layers, n_seqs=n_seqs, n_kv_heads=hkv, max_ctx=max_ctx, type_k=type_k,
-                   type_v=type_v or type_k, tail=tail, sinkhorn_iters=iters)
+                   type_v=type_v or type_k, tail=tail, sinkhorn_iters=iters, tail_f16=tail_f16)
 
 
 def to_dev_bf16(tok_major_bits):
@@ -41,9 +41,10 @@ def storage_bytes(cache):
     return cache.storage.cpu().numpy()
 
 
-def compare_stream(cache, buf, type_, layer, seq, head, which, hist, tail):
+def compare_stream(cache, buf, type_, layer, seq, head, which, hist, tail, ring_bits=None):
     """hist: [n, 128] BF16 bits of one stream.  Quantized sub-pages must equal the oracle's
-    images on every byte of a valid token; tail rows must equal the input bits."""
+    images on every byte of a valid token; tail rows must equal the input bits (or ring_bits,
+    the stored 16-bit rows, for an F16 tail)."""
     n = hist.shape[0]
     st = oracle.stream_state(type_, hist, tail)
     Q = st["Q"]
@@ -61,7 +62,8 @@ def compare_stream(cache, buf, type_, layer, seq, head, which, hist, tail):
     for p in range(keep0, n):
         off, nb = cache.locate(1, layer, seq, 0, head, which, p)
         got = buf[off:off + nb].view(np.uint16)
-        assert np.array_equal(got, hist[p]), (type_, seq, head, which, p)
+        want = hist[p] if ring_bits is None else ring_bits[p]
+        assert np.array_equal(got, want), (type_, seq, head, which, p)
     return Q
 
 

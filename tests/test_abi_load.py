@@ -70,3 +70,14 @@ def test_var_norm_resolves_to_the_kvarn_type():
     with pytest.raises(kvq.KVQError) as e:
         kvq.kvq_cache_bytes(kvq.kvq_default_params(var_norm=2))
     assert e.value.code == kvq.KVQ_E_INVAL
+
+
+def test_tail_format_flag():
+    """tail_f16 takes 0 (BF16 tail) or 1 (F16 tail); the tail format does not change sizes."""
+    from bit_kv_cache_17_b200 import kvq
+
+    a = kvq.kvq_cache_bytes(kvq.kvq_default_params(tail_f16=0))
+    assert kvq.kvq_cache_bytes(kvq.kvq_default_params(tail_f16=1)) == a
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.kvq_cache_bytes(kvq.kvq_default_params(tail_f16=2))
+    assert e.value.code == kvq.KVQ_E_INVAL

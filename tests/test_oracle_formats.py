@@ -54,3 +54,22 @@ def test_bf16_is_nearest_even():
     pick_hi = (dhi < dlo) | ((dhi == dlo) & ((lo & 1) == 1))
     ref = np.where(pick_hi, hi, lo).astype(np.uint16)
     assert np.array_equal(got, ref)
+
+
+def test_every_f16_rounding_of_a_bf16_value_is_a_bf16_value():
+    """The F16 tail reading rests on this: fp16(x) of any BF16 x (all 65 536 patterns, NaN
+    aside) is exactly representable in BF16, so a stream with an F16 tail equals the BF16-tail
+    stream of the rounded rows.  The fp16 cast here is numpy's, independent of the oracle."""
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    x = (h.astype(np.uint32) << 16).view(np.float32)
+    y = x.astype(np.float16).astype(np.float32)  # IEEE round to nearest even, overflow to inf
+    ok = ~np.isnan(x)
+    back = ((y.view(np.uint32) >> 16) << 16).view(np.float32)  # truncation to BF16 loses nothing
+    assert np.array_equal(back[ok], y[ok])
+    # the oracle's helper agrees with numpy, and changes only out-of-range values
+    rows = oracle.f16_tail_rows(h[ok])
+    assert np.array_equal(oracle.bf16_to_f32(rows), y[ok])
+    moved = np.nonzero(oracle.bf16_to_f32(rows) != x[ok])[0]
+    ax = np.abs(x[ok][moved])
+    assert np.all((ax < 2.0**-14) | (ax > 65504.0))
+    assert np.array_equal(oracle.f16_tail_bits(h[ok]), x[ok].astype(np.float16).view(np.uint16))
