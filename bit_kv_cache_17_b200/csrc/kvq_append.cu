@@ -465,19 +465,28 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
       const bool ring = g0 + row < s.n0;
       const int f16r = ring ? L.tail_f16 : 0, rnd = ring ? 0 : L.tail_f16;
       float r[D / 2];  // r[i] = channel 2i + h
+      if (f16r | rnd) {
 #pragma unroll
-      for (int j8 = 0; j8 < D / 8; ++j8) {
-        const uint4 raw = src[j8];
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        for (int j8 = 0; j8 < D / 8; ++j8) {
+          const uint4 raw = src[j8];
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
-          if (f16r | rnd) {
+          for (int u = 0; u < 4; ++u) {
             const float2 xf = ring2f(w[u], f16r);
-            x0 = tail_round(xf.x, rnd);
-            x1 = tail_round(xf.y, rnd);
+            const float x0 = tail_round(xf.x, rnd), x1 = tail_round(xf.y, rnd);
+            r[4 * j8 + u] = h ? __fsub_rn(x0, x1) : __fadd_rn(x0, x1);
           }
-          r[4 * j8 + u] = h ? __fsub_rn(x0, x1) : __fadd_rn(x0, x1);
+        }
+      } else {
+#pragma unroll
+        for (int j8 = 0; j8 < D / 8; ++j8) {
+          const uint4 raw = src[j8];
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+            r[4 * j8 + u] = h ? __fsub_rn(x0, x1) : __fadd_rn(x0, x1);
+          }
         }
       }
       f32x2 rp[D / 4];  // (r[2m], r[2m+1])

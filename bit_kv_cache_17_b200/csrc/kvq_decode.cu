@@ -40,6 +40,7 @@ struct DSeq {
   int32_t cta0;         // first CTA of this sequence
   int32_t part0;        // first partial slot of this sequence
   int64_t n, Q;
+  int64_t qa;           // the uniform quantized splits cover [0, qa); a last split covers [qa, Q)
   int64_t dq, dt;       // first quantized token / ring token written by the preceding kernel
 };
 
@@ -128,56 +129,49 @@ __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
 // One block of Q.K or P.V on the tensor cores with its epilogue on packed fp32:
 //   x += f * (256 * hi + lo)
 // for the two columns of this lane (c0/c2 = hi/lo of column 2tq, c1/c3 = hi/lo of column
-// 2tq+1).  The int32 accumulators start at the bits of 1.5 * 2^23, so each result read as
-// a float is 1.5 * 2^23 + value (exact for |value| < 2^22) and one subtraction recovers it.
+// 2tq+1).  The int32 sums (|value| < 2^22) convert to fp32 exactly.
 __device__ __forceinline__ void mma_s8_fold(f32x2 &x, const uint32_t (&a)[4], uint32_t b0, uint32_t b1, f32x2 f) {
-  const f32x2 bias = 0x4B4000004B400000ull;  // (1.5 * 2^23, 1.5 * 2^23)
   const f32x2 k256 = 0x4380000043800000ull;  // (256, 256)
   asm("{\n"
       " .reg .b32 c0, c1, c2, c3;\n"
+      " .reg .f32 h0, h1, l0, l1;\n"
       " .reg .b64 h, l;\n"
       " mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {c0,c1,c2,c3}, {%1,%2,%3,%4}, {%5,%6}, "
       "{%7,%7,%7,%7};\n"
-      " mov.b64 h, {c0, c1};\n"
-      " mov.b64 l, {c2, c3};\n"
-      " sub.rn.f32x2 h, h, %8;\n"
-      " sub.rn.f32x2 l, l, %8;\n"
-      " fma.rn.f32x2 h, h, %9, l;\n"
-      " fma.rn.f32x2 %0, %10, h, %0;\n"
+      " cvt.rn.f32.s32 h0, c0;\n cvt.rn.f32.s32 h1, c1;\n cvt.rn.f32.s32 l0, c2;\n cvt.rn.f32.s32 l1, c3;\n"
+      " mov.b64 h, {h0, h1};\n"
+      " mov.b64 l, {l0, l1};\n"
+      " fma.rn.f32x2 h, h, %8, l;\n"
+      " fma.rn.f32x2 %0, %9, h, %0;\n"
       "}\n"
       : "+l"(x)
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0x4B400000), "l"(bias), "l"(k256),
-        "l"(f));
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0), "l"(k256), "l"(f));
 }
 
-// Q.K of one block with a 24-bit query: the 16-bit part (rows hi / lo as in mma_s8_fold) and a
-// second MMA for the third limb (rows 0..7; rows 8..15 zero), folded as
-//   x += f * (256 * hi + lo + l3 / 254)
 __device__ __forceinline__ void mma_s8_fold3(f32x2 &x, const uint32_t (&a)[4], const uint32_t (&a3)[2], uint32_t b0,
                                              uint32_t b1, f32x2 f) {
-  const f32x2 bias = 0x4B4000004B400000ull;  // (1.5 * 2^23, 1.5 * 2^23)
   const f32x2 k256 = 0x4380000043800000ull;  // (256, 256)
   const f32x2 k254 = 0x3B8102043B810204ull;  // (1/254, 1/254) rounded to fp32
   asm("{\n"
       " .reg .b32 c0, c1, c2, c3, e0, e1, e2, e3;\n"
+      " .reg .f32 h0, h1, l0, l1, m0, m1;\n"
       " .reg .b64 h, l, m;\n"
       " mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {c0,c1,c2,c3}, {%1,%2,%3,%4}, {%7,%8}, "
       "{%9,%9,%9,%9};\n"
-      " mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {e0,e1,e2,e3}, {%5,%13,%6,%13}, {%7,%8}, "
+      " mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {e0,e1,e2,e3}, {%5,%9,%6,%9}, {%7,%8}, "
       "{%9,%9,%9,%9};\n"
-      " mov.b64 h, {c0, c1};\n"
-      " mov.b64 l, {c2, c3};\n"
-      " mov.b64 m, {e0, e1};\n"
-      " sub.rn.f32x2 h, h, %10;\n"
-      " sub.rn.f32x2 l, l, %10;\n"
-      " sub.rn.f32x2 m, m, %10;\n"
-      " fma.rn.f32x2 h, h, %11, l;\n"
-      " fma.rn.f32x2 h, m, %14, h;\n"
-      " fma.rn.f32x2 %0, %12, h, %0;\n"
+      " cvt.rn.f32.s32 h0, c0;\n cvt.rn.f32.s32 h1, c1;\n cvt.rn.f32.s32 l0, c2;\n cvt.rn.f32.s32 l1, c3;\n"
+      " cvt.rn.f32.s32 m0, e0;\n cvt.rn.f32.s32 m1, e1;\n"
+      " mov.b64 h, {h0, h1};\n"
+      " mov.b64 l, {l0, l1};\n"
+      " mov.b64 m, {m0, m1};\n"
+      " fma.rn.f32x2 h, h, %10, l;\n"
+      " fma.rn.f32x2 h, m, %12, h;\n"
+      " fma.rn.f32x2 %0, %11, h, %0;\n"
       "}\n"
       : "+l"(x)
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a3[0]), "r"(a3[1]), "r"(b0), "r"(b1), "r"(0x4B400000),
-        "l"(bias), "l"(k256), "l"(f), "r"(0), "l"(k254));
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a3[0]), "r"(a3[1]), "r"(b0), "r"(b1), "r"(0),
+        "l"(k256), "l"(f), "l"(k254));
 }
 
 // field s (width W) of each byte of `word`, moved to bits [P, P+W) of the same byte
@@ -1168,8 +1162,15 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   int64_t a, b;
   int64_t nch;
   if (!tail) {
-    a = (int64_t)sp * s.cps_q * CH;
-    b = min(a + (int64_t)s.cps_q * CH, s.Q);
+    if (s.qa < s.Q && sp == s.nsq - 1) {
+      // the tokens an overlapped append rewrites, a split of their own: its warps wait for the
+      // append while the other splits stream, then take one chunk each
+      a = s.qa;
+      b = s.Q;
+    } else {
+      a = (int64_t)sp * s.cps_q * CH;
+      b = min(a + (int64_t)s.cps_q * CH, s.qa);
+    }
   } else {
     a = s.Q + (int64_t)(sp - s.nsq) * s.cps_t * CH;
     b = min(a + (int64_t)s.cps_t * CH, s.n);
@@ -1479,6 +1480,8 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
   // tail token (tensor-core path, 512 bytes) as about twice a quantized one
   const double tbq = (double)token_bytes(c->fam_k, c->bits_k) + token_bytes(c->fam_v, c->bits_v);
   const double tbt = 2.0 * tbq;
+  // the decode overlaps the preceding append only when one launch takes every entry
+  pdl = pdl && seqs.size() <= (size_t)MAXS;
   for (size_t base = 0; base < seqs.size(); base += MAXS) {
     const size_t cnt = std::min<size_t>(MAXS, seqs.size() - base);
     DArgs A{};
@@ -1496,14 +1499,19 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
     A.tickets = reinterpret_cast<uint32_t *>(c->base + c->off_tickets);
     // split plan (min-max greedy): every (sequence, part) with tokens starts with one split
     // per KV head; then, while a whole column of hkv CTAs still fits in one wave, the part
-    // whose splits carry the most work gets one more split
-    std::vector<int> nq(cnt), nt(cnt);
+    // whose splits carry the most work gets one more split.  Behind an overlapped append, the
+    // quantized tokens it rewrites (from the chunk holding dq on) form one more split of
+    // their own, so that the wait for the append holds back only that split's few chunks.
+    std::vector<int> nq(cnt), nt(cnt), nd(cnt);
+    std::vector<int64_t> qa(cnt);
     int used = 0;
     for (size_t i = 0; i < cnt; ++i) {
       const DecodeSeq &d = seqs[base + i];
-      nq[i] = d.Q > 0 ? 1 : 0;
+      qa[i] = pdl && d.dq < d.Q ? (d.dq / CH) * CH : d.Q;
+      nd[i] = qa[i] < d.Q ? 1 : 0;
+      nq[i] = qa[i] > 0 ? 1 : 0;
       nt[i] = d.n > d.Q ? 1 : 0;
-      used += hkv * (nq[i] + nt[i]);
+      used += hkv * (nq[i] + nt[i] + nd[i]);
     }
     // when the entries need more than one wave anyway, plan whole waves
     const int budget = std::max(sms, ((used + sms - 1) / sms) * sms);
@@ -1513,10 +1521,10 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
       double most = 0.0;
       for (size_t i = 0; i < cnt; ++i) {
         const DecodeSeq &d = seqs[base + i];
-        const int64_t nchq = (d.Q + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
-        const double wq = nq[i] ? (double)d.Q * tbq / nq[i] : 0.0;
+        const int64_t nchq = (qa[i] + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
+        const double wq = nq[i] ? (double)qa[i] * tbq / nq[i] : 0.0;
         const double wt = nt[i] ? (double)(d.n - d.Q) * tbt / nt[i] : 0.0;
-        if (wq > most && nq[i] < MAXSQ && nq[i] < nchq) { most = wq; best = (int)i; best_t = false; }
+        if (wq > most && nq[i] + nd[i] < MAXSQ && nq[i] < nchq) { most = wq; best = (int)i; best_t = false; }
         if (wt > most && nt[i] < MAXST && nt[i] < ncht) { most = wt; best = (int)i; best_t = true; }
       }
       if (best < 0) break;
@@ -1531,11 +1539,12 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
       s.row = d.row;
       s.n = d.n;
       s.Q = d.Q;
+      s.qa = qa[i];
       s.dq = d.dq;
       s.dt = d.dt;
-      const int64_t nchq = (d.Q + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
+      const int64_t nchq = (qa[i] + CH - 1) / CH, ncht = (d.n - d.Q + CH - 1) / CH;
       s.cps_q = nq[i] ? (int)((nchq + nq[i] - 1) / nq[i]) : 1;
-      s.nsq = nq[i] ? (int)((nchq + s.cps_q - 1) / s.cps_q) : 0;
+      s.nsq = (nq[i] ? (int)((nchq + s.cps_q - 1) / s.cps_q) : 0) + nd[i];
       s.cps_t = nt[i] ? (int)((ncht + nt[i] - 1) / nt[i]) : 1;
       s.nst = nt[i] ? (int)((ncht + s.cps_t - 1) / s.cps_t) : 0;
       if (s.nsq + s.nst == 0) s.nst = 1;  // empty sequence: one empty split writes zeros
@@ -1554,7 +1563,7 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
       note_launches(2);
       continue;
     }
-    if (dispatch(c->fam_k, c->bits_k, M_FUSED, L, A, st, pdl && seqs.size() <= (size_t)MAXS) != cudaSuccess)
+    if (dispatch(c->fam_k, c->bits_k, M_FUSED, L, A, st, pdl) != cudaSuccess)
       return KVQ_E_CUDA;
     note_launches(1);
   }
