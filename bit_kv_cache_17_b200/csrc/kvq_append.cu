@@ -417,7 +417,9 @@ __device__ __forceinline__ void quant_rows(KvarnSmem &S, uint8_t *sub, const Sub
 // group the append touches (it may be a partial group that grows) and s.b the quantized
 // length Q(n1) after the append; items enumerate (which, group, head) with which = 0 for the
 // first W.total/2 items when K and V are processed by one launch (W.which == 2).
-template <int BITS>
+// TF16: the cache's tail is F16 (a separate instance, so that the BF16 instance is free of
+// the conversions).
+template <int BITS, int TF16>
 __global__ void __launch_bounds__(KV_THREADS, 1)
     k_spill_kvarn(LayerView L, Work W, const __nv_bfloat16 *__restrict__ in_k, const __nv_bfloat16 *__restrict__ in_v,
                   int iters) {
@@ -449,7 +451,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
   if (g0 + GROUP >= Q1) {
     for (int64_t p = s.tw + tid / 16; p < s.n1; p += KV_THREADS / 16) {
       const uint4 *src = reinterpret_cast<const uint4 *>(in + ((s.in_off + (p - s.n0)) * L.hkv + head) * D);
-      reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, which, p))[tid & 15] = bf16x8_to_ring(src[tid & 15], L.tail_f16);
+      reinterpret_cast<uint4 *>(ring_row(L, s.seq, head, which, p))[tid & 15] = bf16x8_to_ring(src[tid & 15], TF16);
     }
   }
 
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
       const uint4 *src = reinterpret_cast<const uint4 *>(src_row(L, s, head, which, g0 + row, in));
       // a ring row as stored; an input row rounded to the tail's format (F16 tails)
       const bool ring = g0 + row < s.n0;
-      const int f16r = ring ? L.tail_f16 : 0, rnd = ring ? 0 : L.tail_f16;
+      const int f16r = ring ? TF16 : 0, rnd = ring ? 0 : TF16;
       float r[D / 2];  // r[i] = channel 2i + h
       if (f16r | rnd) {
 #pragma unroll
@@ -690,18 +692,25 @@ cudaError_t spill_qb(int fam, int bits, const LayerView &L, const Work &W, const
   return cudaErrorInvalidValue;
 }
 
-template <int BITS>
-cudaError_t launch_kvarn_t(const LayerView &L, const Work &W, const __nv_bfloat16 *in_k, const __nv_bfloat16 *in_v,
-                           int iters, cudaStream_t st) {
+template <int BITS, int TF16>
+cudaError_t launch_kvarn_tf(const LayerView &L, const Work &W, const __nv_bfloat16 *in_k, const __nv_bfloat16 *in_v,
+                            int iters, cudaStream_t st) {
   static bool attr_set = false;  // per template instance; the attribute is per function
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_spill_kvarn<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_spill_kvarn<BITS, TF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(KvarnSmem));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_spill_kvarn<BITS><<<(unsigned)W.total, KV_THREADS, sizeof(KvarnSmem), st>>>(L, W, in_k, in_v, iters);
+  k_spill_kvarn<BITS, TF16><<<(unsigned)W.total, KV_THREADS, sizeof(KvarnSmem), st>>>(L, W, in_k, in_v, iters);
   return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_kvarn_t(const LayerView &L, const Work &W, const __nv_bfloat16 *in_k, const __nv_bfloat16 *in_v,
+                           int iters, cudaStream_t st) {
+  return L.tail_f16 ? launch_kvarn_tf<BITS, 1>(L, W, in_k, in_v, iters, st)
+                    : launch_kvarn_tf<BITS, 0>(L, W, in_k, in_v, iters, st);
 }
 
 cudaError_t spill_kvarn(int bits, const LayerView &L, const Work &W, const __nv_bfloat16 *in_k,
