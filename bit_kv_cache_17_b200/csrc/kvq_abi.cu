@@ -296,10 +296,10 @@ int kvq_append_decode(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t
     if (rc) return rc;
     for (const AppendSeq &a : app) c->len[(size_t)layer * c->p.n_seqs + a.seq] = a.n0 + a.n_new;
   }
-  // the decode overlaps the append's last kernel; when that kernel is a small spill it keeps
-  // its SMs, so the decode plans for the others
+  // the decode overlaps the append's last kernel and plans for every SM: the CTAs that wait
+  // for the SMs a small spill still holds are the decode's light ones (its launch order)
   const bool pdl = info.launches > 0;
-  const int budget = info.last_ctas > 0 && info.last_ctas <= c->num_sms / 4 ? c->num_sms - info.last_ctas : 0;
+  const int budget = 0;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
   return launch_decode(c, layer, dec, n_q_heads, q, scale, out, workspace, ws_bytes, st, budget, pdl);
 }

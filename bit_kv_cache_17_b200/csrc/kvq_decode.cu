@@ -1155,7 +1155,19 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   const DSeq &s = A.s[si];
   const int nspl = s.nsq + s.nst;
   const int local = bid - s.cta0;
-  const int head = local / nspl, sp = local % nspl;
+  // CTA order within an entry: the uniform quantized splits of every head first, then the
+  // light ones (the split an overlapped append rewrites, the BF16 tail splits), so that when
+  // a preceding kernel still holds SMs, the CTAs left waiting for them are the light ones
+  const int nreg = s.nsq - (s.qa < s.Q ? 1 : 0);
+  int head, sp;
+  if (local < A.hkv * nreg) {
+    head = local / nreg;
+    sp = local % nreg;
+  } else {
+    const int l2 = local - A.hkv * nreg, nlight = nspl - nreg;
+    head = l2 / nlight;
+    sp = nreg + l2 % nlight;
+  }
   const int G = A.G;
   const bool tail = sp >= s.nsq;
   if (MODE == M_SCORES && tail) return;  // the BF16 tail splits belong to the P.V kernel

@@ -181,10 +181,11 @@ int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_token
  * cache) make these the two halves of every generated token.
  * The decode is launched with programmatic stream serialization behind the append's last
  * kernel: its warps start on pages the append does not touch while the append runs, and
- * wait for it (griddepcontrol.wait) only before the pages and ring rows it rewrites.  When
- * that kernel is a small spill (a one-token step), the decode's split plan leaves the
- * spill's SMs out.  With type_k != type_v the decode follows the append in plain stream
- * order instead.  Requirements beyond the two calls': q must be complete before this call
+ * wait for it (griddepcontrol.wait) only before the pages and ring rows it rewrites, which
+ * form splits of their own.  The decode launches its light CTAs (those splits and the BF16
+ * tail) last, so that the ones left waiting for SMs a one-token spill still holds are
+ * these.  With type_k != type_v the decode follows the append in plain stream order
+ * instead.  Requirements beyond the two calls': q must be complete before this call
  * is issued (it is read while the append runs), and nothing else may be enqueued on `stream`
  * in between (there is nothing in between: this is one call).  Errors: those of the two
  * calls, all checked before anything is launched. */
