@@ -751,7 +751,6 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
       const int64_t Q0 = quantized_len(c, a.n0), Q1 = quantized_len(c, n1);
       if (Q1 <= Q0 || n1 - (Q0 / GROUP) * GROUP > c->ring_cap) ring_fused = false;
     }
-    int spill_ctas = 0;
     for (int which = 0; which < 2; ++which) {
       if (fam[which] == FAM_BF16) continue;
       if (fused && which == 1) continue;
@@ -792,13 +791,8 @@ int launch_append(const kvq_cache *c, int layer, const std::vector<AppendSeq> &s
       if (e != cudaSuccess) return KVQ_E_CUDA;
       note_launches(1);
       ++I.launches;
-      spill_ctas = fam[which] == FAM_KVARN ? (int)W.total : 0;
     }
-    if (ring_fused) {
-      I.last_ctas = spill_ctas;
-      continue;
-    }
-    I.last_ctas = 0;
+    if (ring_fused) continue;
     // 2. ring write of the new rows that stay 16-bit (K and V in one launch when their
     //    types keep the same rows)
     const bool same_keep = fam[0] == fam[1];
