@@ -300,7 +300,7 @@ int kvq_append_decode(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t
   // for the SMs a small spill still holds are the decode's light ones (its launch order)
   const bool pdl = info.launches > 0;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
-  return launch_decode(c, layer, dec, n_q_heads, q, scale, out, workspace, ws_bytes, st, pdl);
+  return launch_decode(c, layer, dec, n_q_heads, q, scale, out, workspace, ws_bytes, st, /*budget_sms=*/0, pdl);
 }
 
 int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_tokens, int32_t n_q_heads,

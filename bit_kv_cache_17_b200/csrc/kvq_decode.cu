@@ -1478,8 +1478,8 @@ size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads) {
 
 int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &seqs, int n_q_heads,
                   const float *q, float scale, float *out, void *ws, size_t ws_bytes, cudaStream_t st,
-                  bool pdl) {
-  const int sms = c->num_sms;
+                  int budget_sms, bool pdl) {
+  const int sms = budget_sms > 0 && budget_sms < c->num_sms ? budget_sms : c->num_sms;
   // K and V of different types: a Q.K kernel of the K type writes the scores, a P.V kernel of
   // the V type reads them (not overlapped with a preceding append)
   const bool mixed = c->p.type_k != c->p.type_v;

@@ -82,12 +82,12 @@ struct DecodeSeq {
   // those kernels (griddepcontrol.wait) before it reads such a token.
   int64_t dq = kNeverDirty, dt = kNeverDirty;
 };
-// pdl: launch with programmatic stream serialization (the previous kernel in the stream must
-// be an append kernel of this library and every token it wrote must be covered by the
-// sequences' dq / dt).  The split plan fills the device's SMs.
+// budget_sms: SMs the split plan may fill (0 = all; every caller passes 0); pdl: launch with
+// programmatic stream serialization (the previous kernel in the stream must be an append
+// kernel of this library and every token it wrote must be covered by the sequences' dq / dt).
 int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &seqs, int n_q_heads,
                   const float *q, float scale, float *out, void *ws, size_t ws_bytes, cudaStream_t st,
-                  bool pdl = false);
+                  int budget_sms = 0, bool pdl = false);
 size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads);
 
 int launch_dequant(const kvq_cache *c, int layer, int seq, int which, int64_t t0, int64_t t1,
