@@ -135,3 +135,26 @@ def test_prefill_chunk_reduces_to_decode_and_to_masked_attention():
             ni = n - n_q + 1 + i
             ref = textbook_attention(q[i], kf[:ni], vf[:ni], scale)
             assert np.max(np.abs(out[i] - ref)) < 1e-10, (t, i)
+
+
+def test_mixed_types_reduce_to_closed_forms():
+    """K and V of different types: the K stream only decides the weights, the V stream only the
+    values.  With every token quantized (tail 0) and a q type, whose tokens are quantized one by
+    one, identical input rows give identical stored rows.  Constant keys then give equal
+    weights, so the output is the mean of the V type's dequantized rows; constant values give
+    that one row whatever the weights."""
+    rng = np.random.default_rng(5)
+    n, G = 700, 3
+    q = rng.standard_normal((G, D)).astype(np.float32)
+    const = np.tile(synth.bf16_bits(rng.standard_normal((1, D)).astype(np.float32)), (n, 1))
+    for tk, tv in (("q8_0", "kvarn2"), ("q4_1", "q3_0"), ("q5_0", "kvarn4")):
+        v = synth.bf16_bits(rng.standard_normal((n, D)).astype(np.float32))
+        out = oracle.decode_head(tk, tv, const, v, 0, q)
+        rows = oracle.dequant(tv, oracle.stream_state(tv, v, 0))
+        assert np.max(np.abs(out - rows.mean(axis=0)[None, :])) < 1e-12
+    for tk, tv in (("kvarn4", "q3_0"), ("kvarn2", "q6_1"), ("q8_0", "q2_0")):
+        k = synth.bf16_bits(rng.standard_normal((n, D)).astype(np.float32))
+        out = oracle.decode_head(tk, tv, k, const, 0, q)
+        rows = oracle.dequant(tv, oracle.stream_state(tv, const, 0))
+        assert np.array_equal(rows, np.tile(rows[:1], (n, 1)))
+        assert np.max(np.abs(out - rows[:1])) < 1e-12
