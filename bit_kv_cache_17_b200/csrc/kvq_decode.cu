@@ -1062,9 +1062,9 @@ __device__ __forceinline__ void warp_wht(float (&v)[4], int lane) {
 
 // Shared memory of the kernel (dynamic): fixed part + per-warp stage area (also used for the
 // warps' accumulators once the chunks are done).
-// What the end of the kernel (CTA combine, ticket, merge) needs of the launch arguments, kept
-// in shared memory from the start: the entry table is indexed at run time, and reading it again
-// after the main loop costs constant-cache misses of about a microsecond each.
+// What the end of the kernel (CTA combine, ticket, merge) needs of the launch arguments,
+// computed once at the start (from the entry table, which is indexed at run time) and kept in
+// shared memory, so that no register holds it across the main loop.
 struct CtaMeta {
   float *rec;        // this (entry, KV head)'s split records: [split][G][PSTRIDE]
   float *out;        // this (entry, KV head)'s output rows: [G][D]
