@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn KV GB/s (% of HBM peak) at 64k ctx; append Mtok/s; vs CPU oracle"
 D = 128
+REPS_APPEND = 5
 
 
 def parse():
@@ -43,6 +44,8 @@ def parse():
     ap.add_argument("--type", default="kvarn4")
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--quick", action="store_true", help="skip the per-type sweep and the append workload")
+    ap.add_argument("--part", default="all", choices=["all", "append"],
+                    help="append: only the batched append workload (for a profiler run)")
     return ap.parse_args()
 
 
@@ -193,6 +196,18 @@ def build_decode_workload(torch, kvq, cfg, type_, layers, tokens_per_layer):
     return cache, kt, vt, P
 
 
+def graph_upload(torch, g):
+    """Uploads an instantiated CUDA graph to the device (cudaGraphUpload on the current
+    stream), so that its first replay inside a timed region does not include the upload."""
+    import ctypes
+
+    rt = ctypes.CDLL("libcudart.so.12")
+    rt.cudaGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    rc = rt.cudaGraphUpload(ctypes.c_void_p(g.raw_cuda_graph_exec()),
+                            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, f"cudaGraphUpload: {rc}"
+
+
 def run_ours(args, ws, rank):
     import torch
 
@@ -234,6 +249,8 @@ def run_ours(args, ws, rank):
                 step(s, out[s])
         graphs.append(g)
     launches = kvq.kvq_launch_count() - launches0
+    for g in graphs:
+        graph_upload(torch, g)
 
     # decode-only graph (state unchanged) for the kernel's own duration and a clock soak
     dec_out = torch.empty((1, hq, D), dtype=torch.float32, device="cuda")
@@ -373,7 +390,8 @@ def run_type_sweep(args, kvq, torch, synth, cfg):
 
 
 def graph_time_us(torch, fn, reps=10):
-    """Mean duration in microseconds of one replay of a CUDA graph of fn()."""
+    """Mean duration in microseconds of one replay of a CUDA graph of fn() (after one
+    untimed replay)."""
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         fn()
@@ -551,15 +569,24 @@ def run_append(args, kvq, torch, synth):
     kin = torch.cat([k[l:l + P] for k, l in zip(ks, Ls)])
     vin = torch.cat([v[l:l + P] for v, l in zip(vs, Ls)])
     torch.cuda.synchronize()
+    # the state before the append: every replay of the captured append starts from it (the
+    # restore is a device copy larger than L2, outside the timed region)
+    snap = cache.storage.clone()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         cache.append(0, list(range(S)), [P] * S, kin, vin)
+    graph_upload(torch, g)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    times = []
+    for _ in range(REPS_APPEND):
+        cache.storage.copy_(snap)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    del snap
+    ms = statistics.median(times)
     assert cache.status() == 0
 
     # batched decode steps: append one token per sequence, then decode all of them
@@ -597,8 +624,15 @@ def run_append(args, kvq, torch, synth):
         q1 = l + P - tail
         staged = q0 - (q0 // 256) * 256
         moved += 2 * hkv * (P * 256 + (tail + staged) * 256 + (q1 - (q0 // 256) * 256) * tb + tail * 256)
+    peaks = load_peaks()
+    gbs = moved / (ms * 1e-3) / 1e9
+    roof = {"kernel": "kvq_append (k_spill_kvarn + k_tail_write)", "bound": "alu (kvarn: WHT + Sinkhorn)",
+            "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+            "ms_per_launch_median": round(ms, 4), "ms_all": [round(x, 4) for x in times],
+            "bytes_per_launch": int(moved), "traffic": traffic_for("spill_bulk_cfg3", "kvarn4")}
     return {"metric": "append Mtok/s", "value": round(S * P / (ms * 1e-3) / 1e6, 2), "unit": "Mtok/s",
-            "ms": round(ms, 4), "GB_per_s": round(moved / (ms * 1e-3) / 1e9, 1), "bytes": int(moved),
+            "ms": round(ms, 4), "GB_per_s": round(gbs, 1), "bytes": int(moved), "roofline": roof,
             "workload": f"{S} sequences, lengths {min(Ls)}..{max(Ls)}, +{P} tokens each in one call, kvarn4, "
                         f"tail {tail}, 8 KV heads x 128", "batched_decode": batched}
 
@@ -636,19 +670,48 @@ def traffic_for(kernel, type_):
 # ---------------------------------------------------------------------------------------
 # the CPU oracle
 
-def _oracle_head_job(job):
-    """One KV head's decode by the oracle (runs in a spawned worker); returns seconds."""
+def _oracle_rows(oracle, type_, hist, tail):
+    """fp64 rows of one stream as the oracle's decode reads them: the quantized region
+    dequantized in the original basis, then the BF16 tail exactly."""
+    st = oracle.stream_state(type_, hist, tail)
+    Q = st["Q"]
+    rows = np.empty((hist.shape[0], D), np.float64)
+    rows[:Q] = oracle.dequant(type_, st, basis=0)
+    rows[Q:] = oracle.bf16_to_f32(hist[Q:])
+    return rows
+
+
+def _oracle_decode_job(job):
+    """One KV head: its state is built untimed, then the oracle's fp64 attention of the G
+    query heads over it is timed (runs in a spawned worker); returns seconds."""
     import oracle
 
     type_, k, v, tail, q = job
+    kr = _oracle_rows(oracle, type_, k, tail)
+    vr = _oracle_rows(oracle, type_, v, tail)
     t0 = time.perf_counter()
-    oracle.decode_head(type_, type_, k, v, tail, q)
+    oracle.attend(q, kr, vr, 1.0 / math.sqrt(D))
+    return time.perf_counter() - t0
+
+
+def _oracle_append_job(job):
+    """One stream of the append sample: the oracle quantizes `n_new` tokens (WHT, Sinkhorn,
+    block quantization of whole groups) behind a BF16 tail; returns seconds."""
+    import oracle
+
+    type_, hist, tail = job
+    t0 = time.perf_counter()
+    oracle.stream_state(type_, hist, tail)
     return time.perf_counter() - t0
 
 
 def cpu_baseline(cfg, type_):
-    """The oracle on the host cores: one decode step at 64k (all KV heads), one head per
-    worker process (spawned, so no worker inherits a CUDA context)."""
+    """The oracle on the host cores, in spawned worker processes (no worker inherits a CUDA
+    context), one KV head (decode) or one stream (append) per job:
+      - decode: one decode step at 64k over a state built before the timed call (the
+        oracle's fp64 attention over its dequantized rows), all KV heads;
+      - append: a sample of the batched append workload, 4096 new tokens of one sequence
+        (8 KV heads x K and V) quantized behind the 1024-token BF16 tail."""
     import multiprocessing as mp
 
     import oracle as calc
@@ -657,20 +720,31 @@ def cpu_baseline(cfg, type_):
     G = cfg["hq"] // hkv
     q = cfg["q"][0, 0]
     cores = len(os.sched_getaffinity(0))
-    nproc = max(1, min(cores, hkv))
-    jobs = [(type_, cfg["k"][h, :n], cfg["v"][h, :n], cfg["tail"], q[h * G:(h + 1) * G]) for h in range(hkv)]
+    nproc = max(1, min(cores, 2 * hkv))
+    dec_jobs = [(type_, cfg["k"][h, :n], cfg["v"][h, :n], cfg["tail"], q[h * G:(h + 1) * G]) for h in range(hkv)]
+    n_new, tail = 4096, cfg["tail"]
+    app_jobs = [(type_, x[h, :n_new + tail], tail) for h in range(hkv) for x in (cfg["k"], cfg["v"])]
     with mp.get_context("spawn").Pool(nproc) as pool:
-        pool.map(_oracle_head_job, jobs[:nproc])  # start the workers (and load the oracle) untimed
+        pool.map(_oracle_append_job, [(type_, cfg["k"][0, :300], 0)] * nproc)  # start the workers untimed
         t0 = time.perf_counter()
-        per_head = pool.map(_oracle_head_job, jobs)
-        wall = time.perf_counter() - t0
+        dec = pool.map(_oracle_decode_job, dec_jobs)
+        dec_wall = time.perf_counter() - t0  # includes the untimed state builds: not used
+        t0 = time.perf_counter()
+        app = pool.map(_oracle_append_job, app_jobs)
+        app_wall = time.perf_counter() - t0
     b = decode_bytes(calc, type_, n, cfg["tail"], hkv, cfg["hq"])
-    single = b / sum(per_head) / 1e9
-    return {"value": round(b / wall / 1e9, 5), "unit": "GB/s", "cores": nproc, "kind": "oracle",
-            "single_thread_value": round(single, 5),
-            "sample": f"one decode step at context {n} ({type_}, {hkv} KV heads, {cfg['hq']} query heads), one KV "
-                      f"head per worker process on {nproc} of {cores} host cores, {wall:.1f} s wall, "
-                      f"{sum(per_head):.1f} s CPU; the oracle rebuilds each stream's state from BF16 in the call"}
+    dec_cpu = sum(dec)
+    par = min(nproc, hkv)
+    dec_par_s = max(dec) if par >= hkv else dec_cpu / par
+    return {"value": round(b / dec_par_s / 1e9, 4), "unit": "GB/s", "cores": par, "kind": "oracle",
+            "single_thread_value": round(b / dec_cpu / 1e9, 4),
+            "sample": f"decode: one step at context {n} ({type_}, {hkv} KV heads, {cfg['hq']} query heads), "
+                      f"state built untimed, one KV head per worker on {par} of {cores} host cores "
+                      f"({dec_cpu:.2f} s CPU in attention); append: {n_new} new tokens of one sequence "
+                      f"(8 KV heads x K/V, behind a {tail}-token tail), one stream per worker",
+            "append": {"value": round(n_new / app_wall / 1e6, 5), "unit": "Mtok/s", "cores": nproc,
+                       "single_thread_value": round(n_new / sum(app) / 1e6, 6),
+                       "seconds_cpu": round(sum(app), 2), "seconds_wall": round(app_wall, 2)}}
 
 
 def run_reference(args, ws, rank):
@@ -710,6 +784,47 @@ def run_reference(args, ws, rank):
             "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def compact(x, digits=4):
+    """Floats rounded to `digits` significant digits, recursively."""
+    if isinstance(x, float):
+        return float(f"{x:.{digits}g}")
+    if isinstance(x, dict):
+        return {k: compact(v, digits) for k, v in x.items()}
+    if isinstance(x, list):
+        return [compact(v, digits) for v in x]
+    return x
+
+
+def summary(result):
+    """The side workloads as roofline fractions of the measured HBM peak (and their times),
+    compact enough to travel with the roofline object."""
+    peak = load_peaks()["hbm_gbs"]
+    out = {}
+    a = result.get("append")
+    if a:
+        out["append_cfg3"] = {"Mtok_per_s": a["value"], "ms": a["ms"], "GB_per_s": a["GB_per_s"],
+                              "frac": a["roofline"]["frac"], "traffic": a["roofline"]["traffic"],
+                              "bytes_per_launch": a["bytes"]}
+        b = a["batched_decode"]
+        out["batched_decode_cfg3"] = {"step_ms": b["ms_per_step"], "decode_us": b["decode_us"],
+                                      "decode_frac": round(b["decode_GB_per_s"] / peak, 4)}
+    t = result.get("per_type_decode_64k")
+    if t:
+        out["decode_64k_frac"] = {k: round(v["GB_per_s"] / peak, 4) for k, v in t.items()}
+        out["decode_64k_us"] = {k: v["decode_us"] for k, v in t.items()}
+    f = result.get("formats_16k")
+    if f:
+        out["decode_16k_frac"] = {k: round(v["GB_per_s"] / peak, 3) for k, v in f["per_format"].items()}
+    p = result.get("page1_shape_240k")
+    if p:
+        out["page1_240k_64_layers"] = {k: {"ms": v["decode_64_layers_ms"], "frac": round(v["GB_per_s"] / peak, 4)}
+                                       for k, v in p["per_type"].items()}
+    c = result.get("prefill_chunk_64k")
+    if c:
+        out["chunk16_64k_us"] = c["us_per_chunk"]
+    return out
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -724,6 +839,11 @@ def main():
 
     from bit_kv_cache_17_b200 import kvq, synth
 
+    if args.part == "append":
+        r = run_append(args, kvq, torch, synth)
+        if rank == 0:
+            print(json.dumps(r))
+        return 0
     result, cfg, cache = run_ours(args, ws, rank)
     del cache
     torch.cuda.empty_cache()
@@ -738,11 +858,14 @@ def main():
         torch.cuda.empty_cache()
         result["prefill_chunk_64k"] = run_prefill(args, kvq, torch, synth)
         torch.cuda.empty_cache()
-        result["quality"] = run_quality(args, kvq, torch, synth)
+        result["quality"] = compact(run_quality(args, kvq, torch, synth))
+        result["roofline"]["others"] = summary(result)
     if rank == 0 and ws == 1:
         result["cpu_baseline"] = cpu_baseline(cfg, args.type)
     elif rank == 0:
         result["cpu_baseline"] = None
+    if "quality" in result:  # the long side report goes last on the line
+        result["quality"] = result.pop("quality")
     if ws > 1:
         import torch.distributed as dist
 

@@ -103,6 +103,13 @@ size_t plan(kvq_cache *c) {
 
 namespace kvq {
 static std::atomic<uint64_t> g_launches{0};
+
+int check_device(const kvq_cache *c) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_E_CUDA;
+  return dev == c->device ? KVQ_OK : KVQ_E_INVAL;
+}
+
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 LayerView layer_view(const kvq_cache *c, int layer) {
@@ -112,6 +119,7 @@ LayerView layer_view(const kvq_cache *c, int layer) {
   L.ptab = reinterpret_cast<const int32_t *>(c->base + c->off_ptab);
   L.status = reinterpret_cast<int32_t *>(c->base + c->off_status);
   L.max_pages = c->max_pages;
+  L.n_phys = (int64_t)c->p.n_seqs * c->max_pages;
   L.page_bytes = c->page_bytes;
   L.ring_cap = c->ring_cap;
   L.hkv = c->p.n_kv_heads;
@@ -238,7 +246,9 @@ int kvq_append(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_i
   if (rows == 0) return KVQ_OK;
   if (!k_bf16 || !v_bf16) return KVQ_E_INVAL;
   if (!aligned16(k_bf16) || !aligned16(v_bf16)) return KVQ_E_ALIGN;
-  int rc = launch_append(c, layer, seqs, k_bf16, v_bf16, reinterpret_cast<cudaStream_t>(stream));
+  int rc = check_device(c);
+  if (rc) return rc;
+  rc = launch_append(c, layer, seqs, k_bf16, v_bf16, reinterpret_cast<cudaStream_t>(stream));
   if (rc) return rc;
   for (const AppendSeq &a : seqs) c->len[(size_t)layer * c->p.n_seqs + a.seq] = a.n0 + a.n_new;
   return KVQ_OK;
@@ -289,6 +299,7 @@ int kvq_append_decode(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t
   }
   if (rows > 0 && (!k_bf16 || !v_bf16)) return KVQ_E_INVAL;
   if (rows > 0 && (!aligned16(k_bf16) || !aligned16(v_bf16))) return KVQ_E_ALIGN;
+  if (const int rc = check_device(c)) return rc;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   AppendInfo info;
   if (rows > 0) {
@@ -324,6 +335,7 @@ int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_token
     const int64_t ni = n - n_q_tokens + 1 + i;
     entries.push_back({seq, i, ni, ni < Q ? ni : Q});
   }
+  if (const int rc = check_device(c)) return rc;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
   return launch_decode(c, layer, entries, n_q_heads, q, scale, out, workspace, ws_bytes,
                        reinterpret_cast<cudaStream_t>(stream));
@@ -348,6 +360,7 @@ int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *
     int64_t n = c->len[(size_t)layer * c->p.n_seqs + s];
     seqs.push_back({s, i, n, quantized_len(c, n)});
   }
+  if (const int rc = check_device(c)) return rc;
   float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
   return launch_decode(c, layer, seqs, n_q_heads, q, scale, out, workspace, ws_bytes,
                        reinterpret_cast<cudaStream_t>(stream));
@@ -362,6 +375,7 @@ int kvq_dequant(kvq_cache *c, int32_t layer, int32_t seq, int32_t which, int64_t
   if (t1 == t0) return KVQ_OK;
   if (!out) return KVQ_E_INVAL;
   if (!aligned16(out)) return KVQ_E_ALIGN;
+  if (const int rc = check_device(c)) return rc;
   return launch_dequant(c, layer, seq, which, t0, t1, basis, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -391,6 +405,19 @@ int kvq_locate(const kvq_cache *c, int32_t kind, int32_t layer, int32_t seq, int
     *bytes = which ? c->lv.bytes : c->lk.bytes;
     return KVQ_OK;
   }
+  if (kind == 3) {
+    // tickets are indexed by (entry of a decode launch, KV head); `seq` is the entry here
+    if (seq >= std::max<int32_t>(c->p.n_seqs, kDecodeEntriesPerLaunch)) return KVQ_E_INVAL;
+    *offset = c->off_tickets + sizeof(uint32_t) * ((size_t)seq * c->p.n_kv_heads + head);
+    *bytes = sizeof(uint32_t);
+    return KVQ_OK;
+  }
+  if (kind == 2) {
+    if (page < 0 || page >= c->max_pages) return KVQ_E_INVAL;
+    *offset = c->off_ptab + sizeof(int32_t) * ((size_t)seq * c->max_pages + page);
+    *bytes = sizeof(int32_t);
+    return KVQ_OK;
+  }
   if (kind == 1) {
     if (c->ring_cap == 0 || token < 0) return KVQ_E_INVAL;
     *offset = c->off_ring + c->layer_ring_bytes * layer +
@@ -404,6 +431,7 @@ int kvq_locate(const kvq_cache *c, int32_t kind, int32_t layer, int32_t seq, int
 
 int kvq_get_status(kvq_cache *c, kvq_stream_t stream) {
   if (!c) return KVQ_E_INVAL;
+  if (const int rc = check_device(c)) return rc;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return KVQ_E_CUDA;
   int32_t st = 0;
   if (cudaMemcpy(&st, c->base + c->off_status, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess)

@@ -110,8 +110,9 @@ struct LayerView {
   uint8_t *pages;        // this layer's page pool
   uint8_t *ring;         // this layer's BF16 ring
   const int32_t *ptab;   // page table [n_seqs * max_pages] -> physical page
-  int32_t *status;       // device status word
+  int32_t *status;       // device status word (KVQ_STATUS_* bits)
   int64_t max_pages;
+  int64_t n_phys;        // physical pages of this layer's pool (n_seqs * max_pages)
   int64_t page_bytes;
   int64_t ring_cap;      // R (rows per ring), 0 if no ring
   int32_t hkv;
@@ -120,9 +121,19 @@ struct LayerView {
   int32_t tail_f16;      // the ring holds F16 rows (else BF16)
 };
 
+// Device status word bits (read and cleared by kvq_get_status): a page-table entry outside the
+// layer's page pool (the access goes to physical page 0 instead, inside the caller's buffer),
+// a merge ticket past the number of splits of its decode.
+constexpr int32_t kStatusPageTable = 1;
+constexpr int32_t kStatusTicket = 2;
+
 __device__ __forceinline__ uint8_t *subpage_ptr(const LayerView &L, int seq, int64_t page, int head,
                                                 int which) {
   int64_t phys = L.ptab[(int64_t)seq * L.max_pages + page];
+  if ((uint64_t)phys >= (uint64_t)L.n_phys) {
+    atomicOr(L.status, kStatusPageTable);
+    phys = 0;
+  }
   return L.pages + phys * L.page_bytes + (int64_t)head * (L.sub_k + L.sub_v) + (which ? L.sub_k : 0);
 }
 

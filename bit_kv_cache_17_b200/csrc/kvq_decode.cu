@@ -1315,6 +1315,8 @@ __global__ void __launch_bounds__(32 * nwarps<FAM, BITS>(), 1) k_decode(LayerVie
   if (tid == 0) {
     __threadfence();
     const unsigned prev = atomicAdd(mt.ticket, 1u);
+    // a ticket past the split count means the counter was not zero when this decode began
+    if (prev >= (unsigned)mt.nspl) atomicOr(L.status, kStatusTicket);
     F.is_last = prev == (unsigned)(mt.nspl - 1);
     if (F.is_last) __threadfence();
   }

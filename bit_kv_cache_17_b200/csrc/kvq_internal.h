@@ -38,6 +38,10 @@ constexpr int kDecodeEntriesPerLaunch = 64;
 // Counts kernel launches (kvq_launch_count).
 void note_launches(int n);
 
+// KVQ_OK when the calling thread's current device is the one the cache was created on,
+// KVQ_E_INVAL when it is another, KVQ_E_CUDA when the runtime cannot tell.
+int check_device(const kvq_cache *c);
+
 // Tokens of a stream kept in the BF16 ring after it holds n tokens: [keep_start, n).
 // qb types keep the tail; kvarn also keeps the rows of its open (partial) group.
 inline int64_t quantized_len(const kvq_cache *c, int64_t n) {

@@ -9,11 +9,12 @@
 //
 // The array lives in this file as a static __device__ variable; every GPU that loads the
 // library holds it (KVQ_NOALLOC_SCRATCH_BYTES) until the process exits.  Host code may not
-// use the variable's name as an address, so the first call on each device looks the device
-// address up once, with that device current, and keeps it.
+// use the variable's name as an address, so every call looks the device address up, with
+// the cache's device current (it checks that first), and passes it to the kernel.  Looking
+// it up each time (cheap once the module is loaded) also stays right after a device reset,
+// when the module is loaded again at another address.
 #include <cuda_runtime.h>
 
-#include <mutex>
 #include <vector>
 
 #include "kvq_internal.h"
@@ -25,22 +26,11 @@ namespace {
 constexpr size_t kScratchBytes = KVQ_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_decode_scratch on the current device (looked up on first use).
+// Device address of g_decode_scratch on the current device.
 int scratch_for_current_device(void **ptr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_E_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return KVQ_E_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return KVQ_E_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *ptr = g_scratch_ptr[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return KVQ_E_CUDA;
+  *ptr = p;
   return KVQ_OK;
 }
 
@@ -57,7 +47,6 @@ extern "C" int kvq_decode_attn_noalloc(kvq_cache *c, int32_t layer, int32_t n_se
   if ((reinterpret_cast<uintptr_t>(q) & 15u) || (reinterpret_cast<uintptr_t>(out) & 15u)) return KVQ_E_ALIGN;
   const size_t need = decode_workspace_bytes(c, n_seqs, n_q_heads);
   if (need > kScratchBytes) return KVQ_E_SIZE;
-  if (c->device < 0) return KVQ_E_INVAL;
   std::vector<char> seen(c->p.n_seqs, 0);
   std::vector<DecodeSeq> seqs;
   for (int i = 0; i < n_seqs; ++i) {
@@ -67,8 +56,11 @@ extern "C" int kvq_decode_attn_noalloc(kvq_cache *c, int32_t layer, int32_t n_se
     const int64_t n = c->len[(size_t)layer * c->p.n_seqs + s];
     seqs.push_back({s, i, n, quantized_len(c, n)});
   }
+  // the scratch array of the cache's own device: the call is rejected when another is current
+  int rc = check_device(c);
+  if (rc) return rc;
   void *scratch = nullptr;
-  const int rc = scratch_for_current_device(&scratch);
+  rc = scratch_for_current_device(&scratch);
   if (rc) return rc;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
   return launch_decode(c, layer, seqs, n_q_heads, q, scale, out, scratch, kScratchBytes,

@@ -38,7 +38,9 @@
  *    inputs, outputs).  The library never allocates device memory.  kvq_cache_destroy
  *    frees only host metadata.
  *  - Pointers marked "device" must be device memory of the current device, 16-byte
- *    aligned (KVQ_E_ALIGN otherwise).
+ *    aligned (KVQ_E_ALIGN otherwise).  Every entry point that touches the device checks,
+ *    before it launches anything, that the calling thread's current device is the one the
+ *    cache was created on: another one gives KVQ_E_INVAL.
  *  - head_dim must be 128; page_tokens and group must be 256 (KVQ_E_UNSUPPORTED).
  *  - GQA: query head h reads KV head h / (n_q_heads / n_kv_heads).
  */
@@ -209,13 +211,23 @@ int kvq_seq_len(const kvq_cache *c, int32_t layer, int32_t seq, int64_t *len);
 int kvq_seq_reset(kvq_cache *c, int32_t seq);
 
 /* Byte offset inside dev_buf of the 256-token sub-page (layer, seq, page, head, which),
- * or of the BF16 ring row holding token `token`, for tests and tools.  kind 0 = sub-page
- * (token ignored), kind 1 = ring row (page ignored).  *bytes receives the region size. */
+ * of the BF16 ring row holding token `token`, of the page-table entry of (seq, page), or
+ * of a decode merge ticket, for tests and tools.  kind 0 = sub-page (token ignored),
+ * kind 1 = ring row (page ignored), kind 2 = page-table entry, an int32 physical page
+ * index shared by all layers, kind 3 = the uint32 merge ticket of KV head `head` of the
+ * decode entry `seq` (the position of a sequence in a decode call's list).  Arguments a
+ * kind does not use are only range-checked.  *bytes receives the region size. */
 int kvq_locate(const kvq_cache *c, int32_t kind, int32_t layer, int32_t seq, int64_t page,
                int32_t head, int32_t which, int64_t token, size_t *offset, size_t *bytes);
 
-/* Synchronizes `stream`, then reads and clears the device status word:
- * KVQ_OK, or KVQ_E_DEVICE if a kernel recorded an internal inconsistency. */
+/* Synchronizes `stream`, then reads and clears the device status word: KVQ_OK, or
+ * KVQ_E_DEVICE if a kernel recorded an inconsistency in the cache buffer since the last
+ * call.  Kernels record (and never trap on):
+ *  - a page-table entry outside the layer's page pool: the access goes to physical page 0
+ *    instead, so nothing outside dev_buf is read or written (the results of that call are
+ *    wrong, the cache buffer having been corrupted);
+ *  - a decode merge ticket that was not zero when the decode began (a corrupted ticket, or
+ *    two decodes of one cache overlapping on the GPU): that decode's output may be stale. */
 int kvq_get_status(kvq_cache *c, kvq_stream_t stream);
 
 /* Human-readable description of the cache (types, tail, bytes); valid until the next
@@ -231,10 +243,15 @@ const char *kvq_strerror(int code);
  * that must not allocate (a possible stall or failure) once it runs.
  *  - The split-K partial results go to one library-owned static device array of
  *    KVQ_NOALLOC_SCRATCH_BYTES (4 MiB) per GPU, held by every GPU that loads the library
- *    until the process exits.  A call whose partials need more (kvq_workspace_bytes for
- *    the same n_seqs / n_q_heads) returns KVQ_E_SIZE and launches nothing.
- *  - The first call on a device looks up the array's device address (with that device
- *    current) and keeps it; make that first call before any stream capture.
+ *    until the process exits.  A call that needs more than the array (kvq_workspace_bytes
+ *    for the same n_seqs / n_q_heads) returns KVQ_E_SIZE and launches nothing.  The need is
+ *    33 792 x n_seqs x n_kv_heads x G bytes of partials (G = n_q_heads / n_kv_heads), plus,
+ *    when type_k != type_v, 4 x n_seqs x n_kv_heads x G x max_ctx (rounded up to 32) bytes
+ *    of scores.  With 8 KV heads and G = 5 that admits 3 sequences of one type, or one
+ *    sequence of a mixed K/V cache with max_ctx <= 17 760.
+ *  - Every call looks the array's device address up with the cache's device current (the
+ *    call is rejected with KVQ_E_INVAL when another device is current); the first call on
+ *    a device may load the library's device code, so make it before any stream capture.
  *  - Every call shares the array and it keeps the last call's contents; nothing in it needs
  *    to start at zero (every partial is written before it is read).  Calls that overlap on
  *    the GPU, on any stream or cache, race on the array: issue them in stream order.
