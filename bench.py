@@ -508,17 +508,18 @@ def run_prefill(args, kvq, torch, synth):
 
 def run_quality(args, kvq, torch, synth):
     """Side report (not a target): attention KL(P_bf16 || P_q) and the relative L2 error of the
-    attention output of a quantized cache against the BF16 cache of the same data, for every
-    type and the tail sizes 0..2048 (context 16384, 8 KV heads, 32 query heads, 4 query
-    draws).  The cache is read back through kvq_dequant (original basis); the attention
-    itself is plain fp32 torch, outside the product path."""
+    attention output of a quantized cache against the BF16 cache of the same data (context
+    16384, 8 KV heads, 32 query heads, 4 query draws).  The cache is read back through
+    kvq_dequant (original basis); the attention itself is plain fp32 torch, outside the
+    product path.  Data sets: the formats workload's AR(1) data with four K outlier channels
+    x20 (every type, tails 0..2048), and two i.i.d. N(0, 1) sets at tails 0 and 1024 for the
+    2- to 4-bit types: with K channels 7 and 63 x16 (the PR1 data) and with no outliers, which
+    separate what the outlier channels do to the rotated types from the types themselves."""
     cfg = synth.config1()
     n, hkv, hq = cfg["n"], cfg["hkv"], cfg["hq"]
     G = hq // hkv
     rng = np.random.default_rng(11)
     q = torch.from_numpy(rng.standard_normal((4, hq, D)).astype(np.float32)).cuda()
-    kt = dev_bf16(torch, synth.token_major(cfg["k"]))
-    vt = dev_bf16(torch, synth.token_major(cfg["v"]))
 
     def attend(kf, vf):  # kf, vf: [n, hkv, D] fp32 -> probabilities [4, hq, n], out [4, hq, D]
         kk = kf.permute(1, 0, 2).repeat_interleave(G, 0)  # [hq, n, D]
@@ -527,27 +528,38 @@ def run_quality(args, kvq, torch, synth):
         p = torch.softmax(s, -1)
         return p, torch.einsum("bhn,hnd->bhd", p, vv)
 
-    p0, o0 = attend(kt.float(), vt.float())
-    lp0 = torch.log(p0.clamp_min(1e-38))
+    def sweep(kbits, vbits, types, tails):
+        kt = dev_bf16(torch, synth.token_major(kbits))
+        vt = dev_bf16(torch, synth.token_major(vbits))
+        p0, o0 = attend(kt.float(), vt.float())
+        lp0 = torch.log(p0.clamp_min(1e-38))
+        out = {}
+        for t in types:
+            row = {}
+            for tail in tails:
+                cache = kvq.KVCache(n_layers=1, n_seqs=1, n_kv_heads=hkv, max_ctx=n, type_k=t, type_v=t, tail=tail)
+                cache.append(0, [0], [n], kt, vt)
+                kf = cache.dequant(0, 0, 0, 0, n)
+                vf = cache.dequant(0, 0, 1, 0, n)
+                p1, o1 = attend(kf, vf)
+                kl = (p0 * (lp0 - torch.log(p1.clamp_min(1e-38)))).sum(-1)  # [4, hq]
+                rel = (o1 - o0).norm(dim=-1) / o0.norm(dim=-1)
+                row[f"T{tail}"] = {"kl_mean": float(kl.mean()), "kl_median": float(kl.median()),
+                                   "out_rel_l2_mean": float(rel.mean())}
+                del cache
+            out[t] = row
+        return out
+
     types = ["q2_0", "q3_0", "q4_0", "q5_0", "q6_0", "q8_0", "q4_1", "q2_1", "q3_1", "q5_1", "q6_1",
              "kvarn2", "kvarn3", "kvarn4", "kvarn5", "kvarn6", "kvarn8"]
-    out = {}
-    for t in types:
-        row = {}
-        for tail in (0, 256, 512, 1024, 2048):
-            cache = kvq.KVCache(n_layers=1, n_seqs=1, n_kv_heads=hkv, max_ctx=n, type_k=t, type_v=t, tail=tail)
-            cache.append(0, [0], [n], kt, vt)
-            kf = cache.dequant(0, 0, 0, 0, n)
-            vf = cache.dequant(0, 0, 1, 0, n)
-            p1, o1 = attend(kf, vf)
-            kl = (p0 * (lp0 - torch.log(p1.clamp_min(1e-38)))).sum(-1)  # [4, hq]
-            rel = (o1 - o0).norm(dim=-1) / o0.norm(dim=-1)
-            row[f"T{tail}"] = {"kl_mean": float(kl.mean()), "kl_median": float(kl.median()),
-                               "out_rel_l2_mean": float(rel.mean())}
-            del cache
-        out[t] = row
-    return {"workload": f"context {n}, {hkv} KV heads, {hq} query heads, 4 query draws (seed 11), data as the "
-                        f"formats workload", "per_type": out}
+    res = {"workload": f"context {n}, {hkv} KV heads, {hq} query heads, 4 query draws (seed 11)",
+           "ar1_outliers20": sweep(cfg["k"], cfg["v"], types, (0, 256, 512, 1024, 2048))}
+    low = ["q2_0", "q3_0", "q4_0", "kvarn2", "kvarn3", "kvarn4"]
+    k, v = synth.kv_iid(np.random.default_rng(12), hkv, n)
+    res["iid_outliers16"] = sweep(k, v, low, (0, 1024))
+    k, v = synth.kv_iid(np.random.default_rng(13), hkv, n, outlier_channels=())
+    res["iid_plain"] = sweep(k, v, low, (0, 1024))
+    return res
 
 
 def run_append(args, kvq, torch, synth):

@@ -327,18 +327,11 @@ int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_token
   if (ws_bytes < decode_workspace_bytes(c, n_q_tokens, n_q_heads)) return KVQ_E_SIZE;
   const int64_t n = c->len[(size_t)layer * c->p.n_seqs + seq];
   if (n_q_tokens > n) return KVQ_E_INVAL;
-  // query i attends to the first n - n_q_tokens + 1 + i tokens of the cache as it is now
-  const int64_t Q = quantized_len(c, n);
-  std::vector<DecodeSeq> entries;
-  entries.reserve(n_q_tokens);
-  for (int i = 0; i < n_q_tokens; ++i) {
-    const int64_t ni = n - n_q_tokens + 1 + i;
-    entries.push_back({seq, i, ni, ni < Q ? ni : Q});
-  }
   if (const int rc = check_device(c)) return rc;
+  // query i attends to the first n - n_q_tokens + 1 + i tokens of the cache as it is now
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
-  return launch_decode(c, layer, entries, n_q_heads, q, scale, out, workspace, ws_bytes,
-                       reinterpret_cast<cudaStream_t>(stream));
+  return launch_chunk(c, layer, seq, n_q_tokens, n_q_heads, q, scale, out, workspace,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *seq_ids,

@@ -94,6 +94,12 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
                   int budget_sms = 0, bool pdl = false);
 size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads);
 
+// Chunk attention (kvq_prefill_attn): n_q query tokens of one sequence, causal within the
+// chunk, 16 query tokens per launch; the workspace holds chunk_workspace_bytes.
+int launch_chunk(const kvq_cache *c, int layer, int seq, int n_q, int n_q_heads, const float *q, float scale,
+                 float *out, void *ws, cudaStream_t st);
+size_t chunk_workspace_bytes(const kvq_cache *c, int n_q_tokens, int n_q_heads);
+
 int launch_dequant(const kvq_cache *c, int layer, int seq, int which, int64_t t0, int64_t t1,
                    int basis, float *out, cudaStream_t st);
 

@@ -3,7 +3,8 @@ oracle's chunk reference: query i sees the first n - n_q + 1 + i tokens of the c
 of the full history (relative L2 <= 1e-3, max abs <= 2e-3 x RMS per query row).
 
 Cases: a chunk inside the BF16 tail; a chunk longer than the tail (the early queries end
-inside the quantized prefix); more than 64 queries (two launches); GQA 5; the BF16 type."""
+inside the quantized prefix); more than 16 queries (several launches); GQA 5; the BF16 type;
+chunks of 64 and 256 queries at context 65536."""
 import numpy as np
 import pytest
 
@@ -45,3 +46,25 @@ def test_prefill_rejects_a_chunk_longer_than_the_sequence():
     with pytest.raises(kvq.KVQError) as e:
         c.prefill_attn(0, 0, q)
     assert e.value.code == kvq.KVQ_E_INVAL
+
+
+@pytest.mark.parametrize("type_,hkv,n_q", [("kvarn4", 2, 64), ("q4_1", 1, 256)])
+def test_prefill_chunk_at_64k_matches_oracle(type_, hkv, n_q):
+    """Long context: a 64k-token cache (1024-token tail) and chunks of 64 and 256 queries, every
+    query row against the oracle (several launches of 16 query tokens, each over the whole
+    quantized prefix)."""
+    th = H.torch()
+    G, n, tail = 5, 65536, 1024
+    rng = np.random.default_rng(n_q)
+    k, v, _ = synth.kv_ar1(rng, hkv, n)
+    c = H.make_cache(type_, hkv, n, tail)
+    H.append(c, 0, [0], [(synth.token_major(k), synth.token_major(v))])
+    q = rng.standard_normal((n_q, hkv * G, 128)).astype(np.float32)
+    out = c.prefill_attn(0, 0, th.from_numpy(q).cuda())
+    th.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    for h in range(hkv):
+        ref = oracle.prefill_head(type_, type_, k[h], v[h], tail, q[:, h * G:(h + 1) * G])
+        for i in range(n_q):
+            H.check_decode(got[i, h * G:(h + 1) * G], ref[i], f"{type_} head {h} query {i}")
+    assert c.status() == 0
