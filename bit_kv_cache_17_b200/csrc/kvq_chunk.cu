@@ -71,12 +71,13 @@ __host__ __device__ inline RawLay raw_lay(int fam, int bits) {
   return r;
 }
 
+constexpr int NS = 2;  // raw chunks in flight (copies run NS - 1 chunks ahead of the dequantization)
 struct Smem {
-  Raw raw[2];                        // double-buffered raw chunks
+  Raw raw[NS];                       // ring of raw chunks
   __half kt[2][CH * TS];             // K-hat hi / lo, [token][channel]
   __half vt[2][CH * TS];             // V-hat hi / lo, [token][channel]
   __half qt[2][MAXR * TS];           // the rows' q'' hi / lo, [row][channel]
-  alignas(16) float qr[MAXR * D];    // the rows' q' (rotated, scaled by qscale), fp32
+  alignas(16) float qr[MAXR * D];    // the rows' q' (rotated for quantized K, scaled by qscale)
   float tk[CH], tv[CH];              // token scales of the chunk (1 for non-kvarn / 16-bit rows)
   alignas(16) __half ck[2][D];       // K / V channel scales of a page (kvarn), by page parity: a
   alignas(16) __half cv[2][D];       // copy one chunk ahead may belong to the next page
@@ -189,9 +190,11 @@ __device__ __forceinline__ void copy_chunk(const LayerView &L, const CArgs &A, i
   }
 }
 
-// One side (K or V) of a quantized chunk: token i, channels 32 blk .. 32 blk + 31 (thread =
-// (token, block)): value = code * d (+ m), times the channel scale c for kvarn V; stored as
-// f16 hi / lo.  A token past the split (ok false) is stored as zeros (its bytes are stale).
+// One side (K or V) of a quantized chunk, by single codes (any type): token i, channels
+// 32 blk .. 32 blk + 31 (thread = (token, block)): value = code * d (+ m) (the kvarn channel
+// scales are applied elsewhere: to the query for K, to the accumulator for V), computed in fp32
+// and stored as f16 hi / lo.  A token past the split (ok false) is stored as zeros (its bytes
+// are stale).
 template <int WHICH, int FAM, int BITS>
 __device__ __forceinline__ void dequant_q(const uint8_t *raw, const __half *cs, __half *hi, __half *lo, int tok,
                                           int blk, bool ok) {
@@ -209,15 +212,146 @@ __device__ __forceinline__ void dequant_q(const uint8_t *raw, const __half *cs, 
     for (int u = 0; u < 2; ++u) {
       const int ch = 32 * blk + e + u;
       const uint32_t f = WHICH == 0 ? k_field<BITS>(tokp, ch) : v_field<BITS>(quad, tok & 3, ch);
-      float val = fmaf((float)code_value<FAM, BITS>(f), d, m);
-      if (WHICH == 1 && FAM == FAM_KVARN) val *= __half2float(cs[ch]);
-      x[u] = ok ? val : 0.f;
+      x[u] = ok ? fmaf((float)code_value<FAM, BITS>(f), d, m) : 0.f;
     }
     const __half2 hh = __floats2half2_rn(x[0], x[1]);
     const float2 hf = __half22float2(hh);
     const __half2 ll = __floats2half2_rn(x[0] - hf.x, x[1] - hf.y);
     *reinterpret_cast<__half2 *>(h + e) = hh;
     *reinterpret_cast<__half2 *>(l + e) = ll;
+  }
+}
+
+// ---- word-level dequantization of symmetric codes (qN_0, kvarn) ------------------------------
+//
+// A 32-bit word of a code plane holds four b-bit fields (one per byte, after a shift and a
+// mask); xor with 2^(b-1) in every byte turns b-bit two's complement codes into c + 2^(b-1), and
+// pairing each byte with 0x64 gives the f16 value 1024 + c + 2^(b-1), exactly; one f16
+// subtraction leaves the code c.  hi = RN(c d) and lo = c d - hi (one fused multiply-add) are
+// f16 again (exact: c d has at most 19 significant bits).
+
+template <int W>
+__device__ __forceinline__ constexpr uint32_t bytes_mask() {
+  return ((1u << W) - 1u) * 0x01010101u;
+}
+
+// codes + 2^(b-1) of 4 consecutive fields as bytes -> 2 f16 pairs of the codes, times d (hi, lo)
+template <int BITS>
+__device__ __forceinline__ void fields_to_half(uint32_t u, __half2 d2, uint32_t &h01, uint32_t &h23, uint32_t &l01,
+                                               uint32_t &l23) {
+  const uint32_t v = u ^ (0x01010101u << (BITS - 1));
+  const __half2 off = __float2half2_rn((float)(1024 + (1 << (BITS - 1))));
+  const uint32_t a = __byte_perm(v, 0x64646464u, 0x5140), b = __byte_perm(v, 0x64646464u, 0x5342);
+  const __half2 c01 = __hsub2(*reinterpret_cast<const __half2 *>(&a), off);
+  const __half2 c23 = __hsub2(*reinterpret_cast<const __half2 *>(&b), off);
+  const __half2 x01 = __hmul2(c01, d2), x23 = __hmul2(c23, d2);
+  const __half2 r01 = __hfma2(c01, d2, __hneg2(x01)), r23 = __hfma2(c23, d2, __hneg2(x23));
+  h01 = h2u(x01);
+  h23 = h2u(x23);
+  l01 = h2u(r01);
+  l23 = h2u(r23);
+}
+
+// K: token tok, block blk (thread); channels 32 blk + 4 jj + k are byte k of word (jj / F, blk)
+template <int BITS>
+__device__ __forceinline__ void dequant_k_fast(const uint8_t *raw, __half *hi, __half *lo, int tok, int blk, bool ok) {
+  constexpr int WL = plane_lo(BITS), WH = plane_hi(BITS);
+  constexpr int FL = 8 / WL, FH = WH ? 8 / WH : 1;
+  const RawLay rl = raw_lay(FAM_SYM, BITS);
+  const __half dh = ok ? reinterpret_cast<const __half *>(raw + rl.d)[tok * 4 + blk] : __float2half(0.f);
+  const __half2 d2 = __halves2half2(dh, dh);
+  const uint8_t *tp = raw + tok * 16 * BITS;
+  __half *h = hi + tok * TS + 32 * blk, *l = lo + tok * TS + 32 * blk;
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const uint32_t wl = *reinterpret_cast<const uint32_t *>(tp + 16 * (jj / FL) + 4 * blk);
+    uint32_t u = (wl >> ((jj % FL) * WL)) & bytes_mask<WL>();
+    if constexpr (WH > 0) {
+      const uint32_t wh = *reinterpret_cast<const uint32_t *>(tp + 16 * WL + 16 * (jj / FH) + 4 * blk);
+      u |= ((wh >> ((jj % FH) * WH)) & bytes_mask<WH>()) << WL;
+    }
+    uint32_t h01, h23, l01, l23;
+    fields_to_half<BITS>(u, d2, h01, h23, l01, l23);
+    *reinterpret_cast<uint2 *>(h + 4 * jj) = make_uint2(h01, h23);
+    *reinterpret_cast<uint2 *>(l + 4 * jj) = make_uint2(l01, l23);
+  }
+}
+
+// V: quad q, block blk, 8 channels 32 blk + 8 j8 .. + 7 of the quad's 4 tokens (thread).  In a
+// plane of width w the channel 32 blk + e of token k is byte k of word e / F at 16 w blk + 4 (e / F),
+// bits (e % F) w: the thread's channels are the fields of words (8 j8 / F) .. (8 j8 + 7) / F.
+template <int BITS>
+__device__ __forceinline__ void dequant_v_fast(const uint8_t *raw, __half *hi, __half *lo, int q, int blk, int j8,
+                                               int64_t tok_end) {
+  constexpr int WL = plane_lo(BITS), WH = plane_hi(BITS);
+  constexpr int FL = 8 / WL, FH = WH ? 8 / WH : 1;
+  constexpr int NL = 8 / FL, NH = WH ? 8 / FH : 0;  // words of each plane holding the 8 channels
+  const RawLay rl = raw_lay(FAM_SYM, BITS);
+  const uint8_t *qp = raw + q * 64 * BITS;
+  uint32_t wl[NL], wh[NH > 0 ? NH : 1];
+#pragma unroll
+  for (int i = 0; i < NL; ++i) wl[i] = *reinterpret_cast<const uint32_t *>(qp + 16 * WL * blk + 4 * (NL * j8 + i));
+#pragma unroll
+  for (int i = 0; i < NH; ++i) wh[i] = *reinterpret_cast<const uint32_t *>(qp + 64 * WL + 16 * WH * blk + 4 * (NH * j8 + i));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int tok = 4 * q + k;
+    const bool ok = tok < tok_end;
+    const __half dh = ok ? reinterpret_cast<const __half *>(raw + rl.d)[tok * 4 + blk] : __float2half(0.f);
+    const __half2 d2 = __halves2half2(dh, dh);
+    __half *h = hi + tok * TS + 32 * blk + 8 * j8, *l = lo + tok * TS + 32 * blk + 8 * j8;
+    uint32_t u[2];  // fields of channels 0..3 and 4..7 of the group, one per byte
+    if constexpr (BITS == 4) {
+      // byte k of the 4 words, then low nibbles = even channels, high nibbles = odd channels
+      const uint32_t sel = (uint32_t)k | ((uint32_t)(4 + k) << 4);
+      const uint32_t x = __byte_perm(__byte_perm(wl[0], wl[1], sel), __byte_perm(wl[2], wl[3], sel), 0x5410);
+      const uint32_t ev = x & 0x0f0f0f0fu, od = (x >> 4) & 0x0f0f0f0fu;
+      u[0] = __byte_perm(ev, od, 0x5140);
+      u[1] = __byte_perm(ev, od, 0x7362);
+    } else {
+#pragma unroll
+      for (int g4 = 0; g4 < 2; ++g4) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = 4 * g4 + i;
+          uint32_t f = (wl[e / FL] >> (8 * k + (e % FL) * WL)) & ((1u << WL) - 1u);
+          if constexpr (WH > 0) f |= ((wh[e / FH] >> (8 * k + (e % FH) * WH)) & ((1u << WH) - 1u)) << WL;
+          acc |= f << (8 * i);
+        }
+        u[g4] = acc;
+      }
+    }
+#pragma unroll
+    for (int g4 = 0; g4 < 2; ++g4) {
+      uint32_t h01, h23, l01, l23;
+      fields_to_half<BITS>(u[g4], d2, h01, h23, l01, l23);
+      *reinterpret_cast<uint2 *>(h + 4 * g4) = make_uint2(h01, h23);
+      *reinterpret_cast<uint2 *>(l + 4 * g4) = make_uint2(l01, l23);
+    }
+  }
+}
+
+__device__ __forceinline__ void dequant_k_sym(int bits, const uint8_t *raw, __half *hi, __half *lo, int tok, int blk,
+                                              bool ok) {
+  switch (bits) {
+    case 2: dequant_k_fast<2>(raw, hi, lo, tok, blk, ok); break;
+    case 3: dequant_k_fast<3>(raw, hi, lo, tok, blk, ok); break;
+    case 4: dequant_k_fast<4>(raw, hi, lo, tok, blk, ok); break;
+    case 5: dequant_k_fast<5>(raw, hi, lo, tok, blk, ok); break;
+    case 6: dequant_k_fast<6>(raw, hi, lo, tok, blk, ok); break;
+    default: dequant_k_fast<8>(raw, hi, lo, tok, blk, ok); break;
+  }
+}
+__device__ __forceinline__ void dequant_v_sym(int bits, const uint8_t *raw, __half *hi, __half *lo, int q, int blk,
+                                              int j8, int64_t tok_end) {
+  switch (bits) {
+    case 2: dequant_v_fast<2>(raw, hi, lo, q, blk, j8, tok_end); break;
+    case 3: dequant_v_fast<3>(raw, hi, lo, q, blk, j8, tok_end); break;
+    case 4: dequant_v_fast<4>(raw, hi, lo, q, blk, j8, tok_end); break;
+    case 5: dequant_v_fast<5>(raw, hi, lo, q, blk, j8, tok_end); break;
+    case 6: dequant_v_fast<6>(raw, hi, lo, q, blk, j8, tok_end); break;
+    default: dequant_v_fast<8>(raw, hi, lo, q, blk, j8, tok_end); break;
   }
 }
 
@@ -236,8 +370,8 @@ __device__ __forceinline__ void dequant_side(int fam, int bits, const uint8_t *r
 #undef KVQ_DQ
 }
 
-// q'' of the rows (q' times the page's K channel scales for kvarn K) into the f16 tiles; each
-// warp its own 16 rows, lane = 4 channels
+// q'' of this warp's 16 rows into the f16 tiles: q' times the page's K channel scales when ck is
+// given (kvarn K); lane = 4 channels
 __device__ __forceinline__ void build_q_tiles(Smem &S, const __half *ck, int warp, int lane) {
   for (int rr = 0; rr < RT; ++rr) {
     const int row = RT * warp + rr;
@@ -275,16 +409,19 @@ __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
   }
   const int nch = b > a ? (int)((b - a + CH - 1) / CH) : 0;
 
-  // first chunk in flight while the rows are rotated
-  if (nch > 0) copy_chunk(L, A, head, a, true, S.raw[0], S, tid);
-  cp_async_commit();
-
-  // q' of every row (row = qi * G + hd), scaled by softmax scale * log2(e); warp per row
+  // the first NS - 1 chunks in flight (one commit group each) while the query tiles are built
+#pragma unroll 1
+  for (int j = 0; j < NS - 1; ++j) {
+    if (j < nch) copy_chunk(L, A, head, a + (int64_t)j * CH, j == 0, S.raw[j], S, tid);
+    cp_async_commit();
+  }
+  // q' of every row (row = qi * G + hd; rows past R are zero), scaled by softmax scale * log2(e)
+  // and, for a quantized kvarn K, rotated; warp per row
   for (int row = warp; row < MAXR; row += NW) {
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (row < R) {
       const int qi = row / G, hd = row % G;
-      const float4 x = *reinterpret_cast<const float4 *>(A.q + ((int64_t)qi * A.hkv * G + head * G + hd) * D + 4 * lane);
+      const float4 x = __ldg(reinterpret_cast<const float4 *>(A.q + ((int64_t)qi * A.hkv * G + head * G + hd) * D) + lane);
       v[0] = x.x * A.qscale;
       v[1] = x.y * A.qscale;
       v[2] = x.z * A.qscale;
@@ -312,14 +449,15 @@ __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[j][e] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  int64_t cur_page = -1;
+  int64_t cur_page = -1, cur_vpage = -1;
+  const bool kvarn_v = !tail && A.fam_v == FAM_KVARN;
 
   for (int c = 0; c < nch; ++c) {
     const int64_t i0 = a + (int64_t)c * CH;
-    const int buf = c & 1;
-    cp_async_wait<0>();
-    __syncthreads();  // chunk c landed; every thread is done with the tiles of chunk c - 1
-    if (c + 1 < nch) copy_chunk(L, A, head, i0 + CH, false, S.raw[buf ^ 1], S, tid);
+    const int buf = c % NS;
+    cp_async_wait<NS - 2>();
+    __syncthreads();  // chunk c landed; every thread is done with the tiles and raw chunk of c - 1
+    if (c + NS - 1 < nch) copy_chunk(L, A, head, i0 + (NS - 1) * CH, false, S.raw[(c + NS - 1) % NS], S, tid);
     cp_async_commit();
     // new kvarn page: q'' of every row from this page's K channel scales
     const int64_t page = i0 / GROUP;
@@ -327,15 +465,27 @@ __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
       build_q_tiles(S, S.ck[page & 1], warp, lane);
       cur_page = page;
     }
-    // dequantize: thread = (token, block) for K and for V
+    // dequantize: warps 0-3 take K (thread = token, block), warps 4-7 take V (symmetric codes:
+    // thread = quad, block, 8 channels; other types: token, block)
     const Raw &rw = S.raw[buf];
     const int tok = tid >> 3, blk = (tid >> 1) & 3, side = tid & 1;
     if (!tail) {
-      const bool ok = i0 + tok < b;
-      if (side == 0)
-        dequant_side<0>(A.fam_k, A.bits_k, rw.k, S.ck[page & 1], S.kt[0], S.kt[1], tok, blk, ok);
-      else
-        dequant_side<1>(A.fam_v, A.bits_v, rw.v, S.cv[page & 1], S.vt[0], S.vt[1], tok, blk, ok);
+      if (tid < 128) {
+        const int tk = tid >> 2, bk = tid & 3;
+        const bool ok = i0 + tk < b;
+        if (A.fam_k != FAM_ASYM)
+          dequant_k_sym(A.bits_k, rw.k, S.kt[0], S.kt[1], tk, bk, ok);
+        else
+          dequant_side<0>(A.fam_k, A.bits_k, rw.k, nullptr, S.kt[0], S.kt[1], tk, bk, ok);
+      } else {
+        const int t = tid - 128;
+        if (A.fam_v != FAM_ASYM) {
+          dequant_v_sym(A.bits_v, rw.v, S.vt[0], S.vt[1], t >> 4, (t >> 2) & 3, t & 3, b - i0);
+        } else {
+          const int tv = t >> 2, bv = t & 3;
+          dequant_side<1>(A.fam_v, A.bits_v, rw.v, nullptr, S.vt[0], S.vt[1], tv, bv, i0 + tv < b);
+        }
+      }
       if (tid < CH) {
         const bool ok = i0 + tid < b;
         S.tk[tid] = !ok ? 0.f
@@ -373,6 +523,22 @@ __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
     }
     __syncthreads();
     if (!active) continue;
+    // kvarn V: the accumulator carries the channel scales of the current page; a new page
+    // rescales it by c_old / c_new (V-hat holds code * d only)
+    if (kvarn_v && page != cur_vpage) {
+      if (cur_vpage >= 0) {
+#pragma unroll
+        for (int jn = 0; jn < 16; ++jn)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int ch = 8 * jn + 2 * tq + e;
+            const float r = __half2float(S.cv[cur_vpage & 1][ch]) / __half2float(S.cv[page & 1][ch]);
+            o[jn][e] *= r;
+            o[jn][2 + e] *= r;
+          }
+      }
+      cur_vpage = page;
+    }
 
     // ---- S = Q.K-hat: 4 n-tiles of 8 tokens, 8 k-steps of 16 channels; hi.hi + lo.hi + hi.lo
     float s[4][4];
@@ -479,6 +645,16 @@ __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
     }
   }
   cp_async_wait<0>();
+  if (kvarn_v && active && cur_vpage >= 0) {
+#pragma unroll
+    for (int jn = 0; jn < 16; ++jn)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float cj = __half2float(S.cv[cur_vpage & 1][8 * jn + 2 * tq + e]);
+        o[jn][e] *= cj;
+        o[jn][2 + e] *= cj;
+      }
+  }
 
   // ---- this split's record of rows r0 and r1: m, l (summed over the 4 lanes of a row), acc
   l0 += __shfl_xor_sync(FULL, l0, 1);
