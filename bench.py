@@ -44,8 +44,9 @@ def parse():
     ap.add_argument("--type", default="kvarn4")
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--quick", action="store_true", help="skip the per-type sweep and the append workload")
-    ap.add_argument("--part", default="all", choices=["all", "append"],
-                    help="append: only the batched append workload (for a profiler run)")
+    ap.add_argument("--part", default="all", choices=["all", "append", "prefill"],
+                    help="append / prefill: only the batched append or the chunk-attention workload "
+                         "(for a profiler run)")
     return ap.parse_args()
 
 
@@ -481,7 +482,7 @@ def run_page1_shape(args, kvq, torch, synth):
 def run_prefill(args, kvq, torch, synth):
     """Chunk attention (kvq_prefill_attn): a 64k-context kvarn4 cache (the headline data) takes
     a chunk of 16 new tokens, whose 16 queries then attend causally; timed in a CUDA graph
-    cycling layer caches.  One entry per query row: each row reads its whole prefix."""
+    cycling layer caches.  Each 32-token piece of the cache is read once for all query rows."""
     calc = LibCalc(kvq)
     cfg = synth.config2()
     n, hkv, hq, tail = cfg["n"], cfg["hkv"], cfg["hq"], cfg["tail"]
@@ -851,8 +852,8 @@ def main():
 
     from bit_kv_cache_17_b200 import kvq, synth
 
-    if args.part == "append":
-        r = run_append(args, kvq, torch, synth)
+    if args.part in ("append", "prefill"):
+        r = (run_append if args.part == "append" else run_prefill)(args, kvq, torch, synth)
         if rank == 0:
             print(json.dumps(r))
         return 0
