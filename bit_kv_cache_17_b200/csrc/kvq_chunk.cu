@@ -30,11 +30,14 @@ namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int CH = 32;               // tokens per chunk
-constexpr int NQ = 16;               // query tokens per launch
-constexpr int RT = 16;               // rows per row tile (one warp)
-constexpr int MAXR = NQ * MAX_G;     // 128 rows
-constexpr int NW = MAXR / RT;        // 8 warps
+constexpr int NQ = 16;               // query tokens per launch (at most MAXR / G)
+constexpr int RT = 16;               // rows per row tile (one consumer warp)
+constexpr int NC = 5;                // consumer warps: Q.K, softmax and P.V of one row tile each
+constexpr int NP = 3;                // producer warps: copies and dequantization
+constexpr int MAXR = NC * RT;        // 80 rows per launch
+constexpr int NW = NP + NC;          // 8 warps
 constexpr int NT = 32 * NW;          // 256 threads
+constexpr int NPT = 32 * NP;         // producer threads
 constexpr int TS = D + 8;            // padded f16 row stride of the shared tiles (272 B)
 constexpr int MAXSPL = 64;           // splits per KV head
 constexpr int PSTRIDE = 4 + D;       // floats per partial record: m, l, 2 pad, acc[128]
@@ -71,14 +74,17 @@ __host__ __device__ inline RawLay raw_lay(int fam, int bits) {
   return r;
 }
 
-constexpr int NS = 2;  // raw chunks in flight (copies run NS - 1 chunks ahead of the dequantization)
-struct Smem {
-  Raw raw[NS];                       // ring of raw chunks
+constexpr int NS = 3;  // raw chunks in the producers' ring (copies run two chunks ahead)
+struct Tiles {
   __half kt[2][CH * TS];             // K-hat hi / lo, [token][channel]
   __half vt[2][CH * TS];             // V-hat hi / lo, [token][channel]
+  float tk[CH], tv[CH];              // token scales of the chunk (1 for non-kvarn / 16-bit rows)
+};
+struct Smem {
+  Raw raw[NS];                       // ring of raw chunks
+  Tiles tile[2];                     // dequantized chunks, double-buffered between the roles
   __half qt[2][MAXR * TS];           // the rows' q'' hi / lo, [row][channel]
   alignas(16) float qr[MAXR * D];    // the rows' q' (rotated for quantized K, scaled by qscale)
-  float tk[CH], tv[CH];              // token scales of the chunk (1 for non-kvarn / 16-bit rows)
   alignas(16) __half ck[2][D];       // K / V channel scales of a page (kvarn), by page parity: a
   alignas(16) __half cv[2][D];       // copy one chunk ahead may belong to the next page
 };
@@ -156,6 +162,7 @@ __device__ __forceinline__ void warp_wht(float (&v)[4], int lane) {
 // the page's parity.
 __device__ __forceinline__ void copy_chunk(const LayerView &L, const CArgs &A, int head, int64_t i0, bool first,
                                            Raw &r, Smem &S, int tid) {
+  constexpr int NT = NPT;  // the producer threads issue the copies
   if (i0 < A.Q) {
     const int64_t page = i0 / GROUP;
     const int tip0 = (int)(i0 % GROUP);
@@ -390,6 +397,76 @@ __device__ __forceinline__ void build_q_tiles(Smem &S, const __half *ck, int war
   }
 }
 
+// named barriers between the roles: FULL[b] (producers arrive when tile buffer b holds a
+// chunk, consumers wait), EMPTY[b] (consumers arrive when done with it, producers wait), and
+// one among the producers
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ void bar_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+constexpr int BAR_FULL = 1, BAR_EMPTY = 3, BAR_PROD = 5;
+
+// Producer side of chunk c: dequantize the raw chunk into tile buffer T (unit u of 256:
+// quantized K (token, block), quantized V (quad, block, 8 channels) or (token, block) for qb_1,
+// 16-bit rows (token, 32 channels, side)).
+__device__ __forceinline__ void produce_tile(const LayerView &L, const CArgs &A, const Raw &rw, Tiles &T, bool tail,
+                                             int64_t i0, int64_t b, int ptid) {
+  for (int u = ptid; u < 256; u += NPT) {
+    if (!tail) {
+      if (u < 128) {
+        const int tk = u >> 2, bk = u & 3;
+        const bool ok = i0 + tk < b;
+        if (A.fam_k != FAM_ASYM)
+          dequant_k_sym(A.bits_k, rw.k, T.kt[0], T.kt[1], tk, bk, ok);
+        else
+          dequant_side<0>(A.fam_k, A.bits_k, rw.k, nullptr, T.kt[0], T.kt[1], tk, bk, ok);
+      } else {
+        const int t = u - 128;
+        if (A.fam_v != FAM_ASYM) {
+          dequant_v_sym(A.bits_v, rw.v, T.vt[0], T.vt[1], t >> 4, (t >> 2) & 3, t & 3, b - i0);
+        } else {
+          const int tv = t >> 2, bv = t & 3;
+          dequant_side<1>(A.fam_v, A.bits_v, rw.v, nullptr, T.vt[0], T.vt[1], tv, bv, i0 + tv < b);
+        }
+      }
+    } else {
+      // 16-bit rows: rows past the end are zero
+      const int tok = u >> 3, blk = (u >> 1) & 3, side = u & 1;
+      const bool ok = i0 + tok < b;
+      const uint8_t *src = (side ? rw.v : rw.k) + 256 * tok + 64 * blk;
+      __half *h = (side ? T.vt[0] : T.kt[0]) + tok * TS + 32 * blk;
+      __half *l = (side ? T.vt[1] : T.kt[1]) + tok * TS + 32 * blk;
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const uint32_t w = ok ? *reinterpret_cast<const uint32_t *>(src + 2 * e) : 0u;
+        float x0, x1;
+        if (L.tail_f16) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
+          x0 = f.x;
+          x1 = f.y;
+        } else {
+          x0 = __uint_as_float(w << 16);
+          x1 = __uint_as_float(w & 0xffff0000u);
+        }
+        const __half2 hh = __floats2half2_rn(x0, x1);
+        const float2 hf = __half22float2(hh);
+        *reinterpret_cast<__half2 *>(h + e) = hh;
+        *reinterpret_cast<__half2 *>(l + e) = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+      }
+    }
+  }
+  if (ptid < CH) {
+    const bool ok = i0 + ptid < b;
+    float tkv = ok ? 1.f : 0.f, tvv = tkv;
+    if (!tail && ok && A.fam_k == FAM_KVARN)
+      tkv = __half2float(reinterpret_cast<const __half *>(rw.k + raw_lay(A.fam_k, A.bits_k).t)[ptid]);
+    if (!tail && ok && A.fam_v == FAM_KVARN)
+      tvv = __half2float(reinterpret_cast<const __half *>(rw.v + raw_lay(A.fam_v, A.bits_v).t)[ptid]);
+    T.tk[ptid] = tkv;
+    T.tv[ptid] = tvv;
+  }
+}
+
 __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem &S = *reinterpret_cast<Smem *>(smem_raw);
@@ -408,12 +485,15 @@ __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
     b = min(a + (int64_t)A.cps_t * CH, A.n);
   }
   const int nch = b > a ? (int)((b - a + CH - 1) / CH) : 0;
+  const bool producer = warp < NP;
 
-  // the first NS - 1 chunks in flight (one commit group each) while the query tiles are built
+  // the producers' first NS - 1 chunks in flight (one commit group each) while q' is computed
+  if (producer) {
 #pragma unroll 1
-  for (int j = 0; j < NS - 1; ++j) {
-    if (j < nch) copy_chunk(L, A, head, a + (int64_t)j * CH, j == 0, S.raw[j], S, tid);
-    cp_async_commit();
+    for (int j = 0; j < NS - 1; ++j) {
+      if (j < nch) copy_chunk(L, A, head, a + (int64_t)j * CH, j == 0, S.raw[j], S, tid);
+      cp_async_commit();
+    }
   }
   // q' of every row (row = qi * G + hd; rows past R are zero), scaled by softmax scale * log2(e)
   // and, for a quantized kvarn K, rotated; warp per row
@@ -435,14 +515,32 @@ __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
     *reinterpret_cast<float4 *>(&S.qr[row * D + 4 * lane]) = make_float4(v[0], v[1], v[2], v[3]);
   }
   __syncthreads();
-  const bool kvarn_k = !tail && A.fam_k == FAM_KVARN;
-  if (!kvarn_k) build_q_tiles(S, nullptr, warp, lane);  // (kvarn K: per page, below)
 
-  // this warp's rows: tile rows g and g + 8; their causal limits
-  const int r0 = RT * warp + g, r1 = r0 + 8;
+  if (producer) {
+    // ---- producers: copies two chunks ahead, dequantization into the tile buffers
+    for (int c = 0; c < nch; ++c) {
+      const int64_t i0 = a + (int64_t)c * CH;
+      const int tb = c & 1;
+      cp_async_wait<NS - 2>();   // this thread's copies of chunk c have landed
+      bar_sync(BAR_PROD, NPT);   // ... every producer's, and every producer is done with chunk c - 1
+      if (c + NS - 1 < nch) copy_chunk(L, A, head, i0 + (NS - 1) * CH, false, S.raw[(c + NS - 1) % NS], S, tid);
+      cp_async_commit();
+      if (c >= 2) bar_sync(BAR_EMPTY + tb, NT);  // the consumers are done with chunk c - 2
+      produce_tile(L, A, S.raw[c % NS], S.tile[tb], tail, i0, b, tid);
+      bar_arrive(BAR_FULL + tb, NT);
+    }
+    cp_async_wait<0>();
+    return;
+  }
+
+  // ---- consumers: warp w' = warp - NP takes rows 16 w' .. 16 w' + 15
+  const int cw = warp - NP;
+  const bool kvarn_k = !tail && A.fam_k == FAM_KVARN;
+  if (!kvarn_k) build_q_tiles(S, nullptr, cw, lane);  // (kvarn K: per page, below)
+  const int r0 = RT * cw + g, r1 = r0 + 8;
   const int64_t lim0 = r0 < R ? A.n - A.nq + 1 + r0 / G : 0;
   const int64_t lim1 = r1 < R ? A.n - A.nq + 1 + r1 / G : 0;
-  const bool active = RT * warp < R;
+  const bool active = RT * cw < R;
   float o[16][4];
 #pragma unroll
   for (int j = 0; j < 16; ++j)
@@ -454,197 +552,140 @@ __global__ void __launch_bounds__(NT, 1) k_chunk(LayerView L, CArgs A) {
 
   for (int c = 0; c < nch; ++c) {
     const int64_t i0 = a + (int64_t)c * CH;
-    const int buf = c % NS;
-    cp_async_wait<NS - 2>();
-    __syncthreads();  // chunk c landed; every thread is done with the tiles and raw chunk of c - 1
-    if (c + NS - 1 < nch) copy_chunk(L, A, head, i0 + (NS - 1) * CH, false, S.raw[(c + NS - 1) % NS], S, tid);
-    cp_async_commit();
-    // new kvarn page: q'' of every row from this page's K channel scales
+    const int tb = c & 1;
+    const Tiles &T = S.tile[tb];
+    bar_sync(BAR_FULL + tb, NT);  // chunk c is in tile buffer tb (and its page scales have landed)
     const int64_t page = i0 / GROUP;
+    // new kvarn page: q'' of this warp's rows from the page's K channel scales
     if (kvarn_k && page != cur_page) {
-      build_q_tiles(S, S.ck[page & 1], warp, lane);
+      build_q_tiles(S, S.ck[page & 1], cw, lane);
+      __syncwarp();
       cur_page = page;
     }
-    // dequantize: warps 0-3 take K (thread = token, block), warps 4-7 take V (symmetric codes:
-    // thread = quad, block, 8 channels; other types: token, block)
-    const Raw &rw = S.raw[buf];
-    const int tok = tid >> 3, blk = (tid >> 1) & 3, side = tid & 1;
-    if (!tail) {
-      if (tid < 128) {
-        const int tk = tid >> 2, bk = tid & 3;
-        const bool ok = i0 + tk < b;
-        if (A.fam_k != FAM_ASYM)
-          dequant_k_sym(A.bits_k, rw.k, S.kt[0], S.kt[1], tk, bk, ok);
-        else
-          dequant_side<0>(A.fam_k, A.bits_k, rw.k, nullptr, S.kt[0], S.kt[1], tk, bk, ok);
-      } else {
-        const int t = tid - 128;
-        if (A.fam_v != FAM_ASYM) {
-          dequant_v_sym(A.bits_v, rw.v, S.vt[0], S.vt[1], t >> 4, (t >> 2) & 3, t & 3, b - i0);
-        } else {
-          const int tv = t >> 2, bv = t & 3;
-          dequant_side<1>(A.fam_v, A.bits_v, rw.v, nullptr, S.vt[0], S.vt[1], tv, bv, i0 + tv < b);
+    if (active) {
+      // kvarn V: the accumulator carries the channel scales of the current page; a new page
+      // rescales it by c_old / c_new (V-hat holds code * d only)
+      if (kvarn_v && page != cur_vpage) {
+        if (cur_vpage >= 0) {
+#pragma unroll
+          for (int jn = 0; jn < 16; ++jn)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int ch = 8 * jn + 2 * tq + e;
+              const float r = __half2float(S.cv[cur_vpage & 1][ch]) / __half2float(S.cv[page & 1][ch]);
+              o[jn][e] *= r;
+              o[jn][2 + e] *= r;
+            }
+        }
+        cur_vpage = page;
+      }
+      // ---- S = Q.K-hat: 4 n-tiles of 8 tokens, 8 k-steps of 16 channels; hi.hi + lo.hi + hi.lo
+      float s[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+      const __half *qh = &S.qt[0][(RT * cw + (lane & 15)) * TS + 8 * (lane >> 4)];
+      const __half *ql = &S.qt[1][(RT * cw + (lane & 15)) * TS + 8 * (lane >> 4)];
+      // B: lanes 0-7 / 8-15 / 16-23 / 24-31 address matrices (tokens 8 nt2 + 0..7, channels
+      // k0 + 0..7), (same tokens, k0 + 8..15), (tokens 8 nt2 + 8.., k0), (tokens 8 nt2 + 8.., k0 + 8)
+      const int brow = (lane & 7) + 8 * (lane >> 4), bcol = 8 * ((lane >> 3) & 1);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t ah[4], al[4];
+        ldsm_x4(ah, qh + 16 * ks);
+        ldsm_x4(al, ql + 16 * ks);
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {  // pairs of n-tiles
+          uint32_t bh[4], bl[4];
+          ldsm_x4(bh, &T.kt[0][(16 * np + brow) * TS + 16 * ks + bcol]);
+          ldsm_x4(bl, &T.kt[1][(16 * np + brow) * TS + 16 * ks + bcol]);
+          mma16(s[2 * np], ah, bh[0], bh[1]);
+          mma16(s[2 * np], al, bh[0], bh[1]);
+          mma16(s[2 * np], ah, bl[0], bl[1]);
+          mma16(s[2 * np + 1], ah, bh[2], bh[3]);
+          mma16(s[2 * np + 1], al, bh[2], bh[3]);
+          mma16(s[2 * np + 1], ah, bl[2], bl[3]);
         }
       }
-      if (tid < CH) {
-        const bool ok = i0 + tid < b;
-        S.tk[tid] = !ok ? 0.f
-                        : (A.fam_k == FAM_KVARN ? __half2float(reinterpret_cast<const __half *>(rw.k + raw_lay(A.fam_k, A.bits_k).t)[tid]) : 1.f);
-        S.tv[tid] = !ok ? 0.f
-                        : (A.fam_v == FAM_KVARN ? __half2float(reinterpret_cast<const __half *>(rw.v + raw_lay(A.fam_v, A.bits_v).t)[tid]) : 1.f);
-      }
-    } else {
-      // 16-bit rows: thread = (token, 32 channels of one side); rows past the end are zero
-      const bool ok = i0 + tok < b;
-      const uint8_t *src = (side ? rw.v : rw.k) + 256 * tok + 64 * blk;
-      __half *h = (side ? S.vt[0] : S.kt[0]) + tok * TS + 32 * blk;
-      __half *l = (side ? S.vt[1] : S.kt[1]) + tok * TS + 32 * blk;
+      // ---- token scales, causal masks, online softmax of rows r0 (c0, c1) and r1 (c2, c3)
+      float cmax0 = -INFINITY, cmax1 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const uint32_t w = ok ? *reinterpret_cast<const uint32_t *>(src + 2 * e) : 0u;
-        float x0, x1;
-        if (L.tail_f16) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
-          x0 = f.x;
-          x1 = f.y;
-        } else {
-          x0 = __uint_as_float(w << 16);
-          x1 = __uint_as_float(w & 0xffff0000u);
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 8 * nt + 2 * tq + e;
+          const int64_t tokg = i0 + t;
+          const float tk = T.tk[t];
+          s[nt][e] = (tokg < lim0 && tokg < b) ? s[nt][e] * tk : -INFINITY;
+          s[nt][2 + e] = (tokg < lim1 && tokg < b) ? s[nt][2 + e] * tk : -INFINITY;
+          cmax0 = fmaxf(cmax0, s[nt][e]);
+          cmax1 = fmaxf(cmax1, s[nt][2 + e]);
         }
-        const __half2 hh = __floats2half2_rn(x0, x1);
-        const float2 hf = __half22float2(hh);
-        *reinterpret_cast<__half2 *>(h + e) = hh;
-        *reinterpret_cast<__half2 *>(l + e) = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+      cmax0 = fmaxf(cmax0, __shfl_xor_sync(FULL, cmax0, 1));
+      cmax0 = fmaxf(cmax0, __shfl_xor_sync(FULL, cmax0, 2));
+      cmax1 = fmaxf(cmax1, __shfl_xor_sync(FULL, cmax1, 1));
+      cmax1 = fmaxf(cmax1, __shfl_xor_sync(FULL, cmax1, 2));
+      const float mn0 = fmaxf(m0, cmax0), mn1 = fmaxf(m1, cmax1);
+      // a row with nothing valid so far keeps m = -inf, weight 0, scale 1
+      const float al0 = mn0 == -INFINITY ? 1.f : exp2_fast(m0 - mn0);
+      const float al1 = mn1 == -INFINITY ? 1.f : exp2_fast(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      float p[4][4], ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          p[nt][e] = mn0 == -INFINITY ? 0.f : exp2_fast(s[nt][e] - mn0);
+          p[nt][2 + e] = mn1 == -INFINITY ? 0.f : exp2_fast(s[nt][2 + e] - mn1);
+          ps0 += p[nt][e];
+          ps1 += p[nt][2 + e];
+        }
+      l0 = fmaf(l0, al0, ps0);
+      l1 = fmaf(l1, al1, ps1);
+      if (__any_sync(FULL, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          o[j][0] *= al0;
+          o[j][1] *= al0;
+          o[j][2] *= al1;
+          o[j][3] *= al1;
+        }
       }
-      if (tid < CH) {
-        S.tk[tid] = i0 + tid < b ? 1.f : 0.f;
-        S.tv[tid] = S.tk[tid];
+      // ---- O += (p t_V) . V-hat: weights as one f16 each (the A fragments of two k-steps of 16
+      //      tokens), V-hat hi and lo through ldmatrix.trans
+      uint32_t pa[2][4];
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        const int ta = 16 * kk + 2 * tq, tb2 = ta + 8;
+        const float va0 = T.tv[ta], va1 = T.tv[ta + 1], vb0 = T.tv[tb2], vb1 = T.tv[tb2 + 1];
+        pa[kk][0] = h2u(__floats2half2_rn(p[2 * kk][0] * va0, p[2 * kk][1] * va1));
+        pa[kk][1] = h2u(__floats2half2_rn(p[2 * kk][2] * va0, p[2 * kk][3] * va1));
+        pa[kk][2] = h2u(__floats2half2_rn(p[2 * kk + 1][0] * vb0, p[2 * kk + 1][1] * vb1));
+        pa[kk][3] = h2u(__floats2half2_rn(p[2 * kk + 1][2] * vb0, p[2 * kk + 1][3] * vb1));
       }
-    }
-    __syncthreads();
-    if (!active) continue;
-    // kvarn V: the accumulator carries the channel scales of the current page; a new page
-    // rescales it by c_old / c_new (V-hat holds code * d only)
-    if (kvarn_v && page != cur_vpage) {
-      if (cur_vpage >= 0) {
+      // B (trans): lanes 0-7 / 8-15 / 16-23 / 24-31 address rows (tokens 16 kk + 0..7, channels
+      // 8 j .. 8 j + 7), (tokens 16 kk + 8.., 8 j ..), (tokens 16 kk + 0..7, 8 (j + 1) ..),
+      // (tokens 16 kk + 8.., 8 (j + 1) ..)
+      const int vrow = (lane & 7) + 8 * ((lane >> 3) & 1), vcol = 8 * (lane >> 4);
 #pragma unroll
-        for (int jn = 0; jn < 16; ++jn)
+      for (int kk = 0; kk < 2; ++kk) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int ch = 8 * jn + 2 * tq + e;
-            const float r = __half2float(S.cv[cur_vpage & 1][ch]) / __half2float(S.cv[page & 1][ch]);
-            o[jn][e] *= r;
-            o[jn][2 + e] *= r;
-          }
-      }
-      cur_vpage = page;
-    }
-
-    // ---- S = Q.K-hat: 4 n-tiles of 8 tokens, 8 k-steps of 16 channels; hi.hi + lo.hi + hi.lo
-    float s[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-    const __half *qh = &S.qt[0][(RT * warp + (lane & 15)) * TS + 8 * (lane >> 4)];
-    const __half *ql = &S.qt[1][(RT * warp + (lane & 15)) * TS + 8 * (lane >> 4)];
-    // B: lanes 0-7 / 8-15 / 16-23 / 24-31 address matrices (tokens 8 nt2 + 0..7, channels k0 + 0..7),
-    // (same tokens, k0 + 8..15), (tokens 8 nt2 + 8.., k0), (tokens 8 nt2 + 8.., k0 + 8)
-    const int brow = (lane & 7) + 8 * (lane >> 4), bcol = 8 * ((lane >> 3) & 1);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t ah[4], al[4];
-      ldsm_x4(ah, qh + 16 * ks);
-      ldsm_x4(al, ql + 16 * ks);
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {  // pairs of n-tiles
-        uint32_t bh[4], bl[4];
-        ldsm_x4(bh, &S.kt[0][(16 * np + brow) * TS + 16 * ks + bcol]);
-        ldsm_x4(bl, &S.kt[1][(16 * np + brow) * TS + 16 * ks + bcol]);
-        mma16(s[2 * np], ah, bh[0], bh[1]);
-        mma16(s[2 * np], al, bh[0], bh[1]);
-        mma16(s[2 * np], ah, bl[0], bl[1]);
-        mma16(s[2 * np + 1], ah, bh[2], bh[3]);
-        mma16(s[2 * np + 1], al, bh[2], bh[3]);
-        mma16(s[2 * np + 1], ah, bl[2], bl[3]);
-      }
-    }
-    // ---- token scales, causal masks, online softmax of rows r0 (c0, c1) and r1 (c2, c3)
-    float cmax0 = -INFINITY, cmax1 = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int t = 8 * nt + 2 * tq + e;
-        const int64_t tokg = i0 + t;
-        const float tk = S.tk[t];
-        s[nt][e] = (tokg < lim0 && tokg < b) ? s[nt][e] * tk : -INFINITY;
-        s[nt][2 + e] = (tokg < lim1 && tokg < b) ? s[nt][2 + e] * tk : -INFINITY;
-        cmax0 = fmaxf(cmax0, s[nt][e]);
-        cmax1 = fmaxf(cmax1, s[nt][2 + e]);
-      }
-    cmax0 = fmaxf(cmax0, __shfl_xor_sync(FULL, cmax0, 1));
-    cmax0 = fmaxf(cmax0, __shfl_xor_sync(FULL, cmax0, 2));
-    cmax1 = fmaxf(cmax1, __shfl_xor_sync(FULL, cmax1, 1));
-    cmax1 = fmaxf(cmax1, __shfl_xor_sync(FULL, cmax1, 2));
-    const float mn0 = fmaxf(m0, cmax0), mn1 = fmaxf(m1, cmax1);
-    // a row with nothing valid so far keeps m = -inf, weight 0, scale 1
-    const float al0 = mn0 == -INFINITY ? 1.f : exp2_fast(m0 - mn0);
-    const float al1 = mn1 == -INFINITY ? 1.f : exp2_fast(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    float p[4][4], ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        p[nt][e] = mn0 == -INFINITY ? 0.f : exp2_fast(s[nt][e] - mn0);
-        p[nt][2 + e] = mn1 == -INFINITY ? 0.f : exp2_fast(s[nt][2 + e] - mn1);
-        ps0 += p[nt][e];
-        ps1 += p[nt][2 + e];
-      }
-    l0 = fmaf(l0, al0, ps0);
-    l1 = fmaf(l1, al1, ps1);
-    if (__any_sync(FULL, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        o[j][0] *= al0;
-        o[j][1] *= al0;
-        o[j][2] *= al1;
-        o[j][3] *= al1;
+        for (int jp = 0; jp < 8; ++jp) {  // pairs of 8-channel n-tiles
+          uint32_t vh[4], vl[4];
+          ldsm_x4_t(vh, &T.vt[0][(16 * kk + vrow) * TS + 16 * jp + vcol]);
+          ldsm_x4_t(vl, &T.vt[1][(16 * kk + vrow) * TS + 16 * jp + vcol]);
+          mma16(o[2 * jp], pa[kk], vh[0], vh[1]);
+          mma16(o[2 * jp], pa[kk], vl[0], vl[1]);
+          mma16(o[2 * jp + 1], pa[kk], vh[2], vh[3]);
+          mma16(o[2 * jp + 1], pa[kk], vl[2], vl[3]);
+        }
       }
     }
-    // ---- O += (p t_V) . V-hat: weights as one f16 each (the A fragments of two k-steps of 16
-    //      tokens), V-hat hi and lo through ldmatrix.trans
-    uint32_t pa[2][4];
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-      const int ta = 16 * kk + 2 * tq, tb = ta + 8;
-      const float va0 = S.tv[ta], va1 = S.tv[ta + 1], vb0 = S.tv[tb], vb1 = S.tv[tb + 1];
-      pa[kk][0] = h2u(__floats2half2_rn(p[2 * kk][0] * va0, p[2 * kk][1] * va1));
-      pa[kk][1] = h2u(__floats2half2_rn(p[2 * kk][2] * va0, p[2 * kk][3] * va1));
-      pa[kk][2] = h2u(__floats2half2_rn(p[2 * kk + 1][0] * vb0, p[2 * kk + 1][1] * vb1));
-      pa[kk][3] = h2u(__floats2half2_rn(p[2 * kk + 1][2] * vb0, p[2 * kk + 1][3] * vb1));
-    }
-    // B (trans): lanes 0-7 / 8-15 / 16-23 / 24-31 address rows (tokens 16 kk + 0..7, channels
-    // 8 j .. 8 j + 7), (tokens 16 kk + 8.., 8 j ..), (tokens 16 kk + 0..7, 8 (j + 1) ..),
-    // (tokens 16 kk + 8.., 8 (j + 1) ..)
-    const int vrow = (lane & 7) + 8 * ((lane >> 3) & 1), vcol = 8 * (lane >> 4);
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-#pragma unroll
-      for (int jp = 0; jp < 8; ++jp) {  // pairs of 8-channel n-tiles
-        uint32_t vh[4], vl[4];
-        ldsm_x4_t(vh, &S.vt[0][(16 * kk + vrow) * TS + 16 * jp + vcol]);
-        ldsm_x4_t(vl, &S.vt[1][(16 * kk + vrow) * TS + 16 * jp + vcol]);
-        mma16(o[2 * jp], pa[kk], vh[0], vh[1]);
-        mma16(o[2 * jp], pa[kk], vl[0], vl[1]);
-        mma16(o[2 * jp + 1], pa[kk], vh[2], vh[3]);
-        mma16(o[2 * jp + 1], pa[kk], vl[2], vl[3]);
-      }
-    }
+    // done with tile buffer tb (the producers wait for it only before chunk c + 2)
+    if (c + 2 < nch) bar_arrive(BAR_EMPTY + tb, NT);
   }
-  cp_async_wait<0>();
   if (kvarn_v && active && cur_vpage >= 0) {
 #pragma unroll
     for (int jn = 0; jn < 16; ++jn)
@@ -751,8 +792,9 @@ int launch_chunk(const kvq_cache *c, int layer, int seq, int n_q, int n_q_heads,
   const int hkv = c->p.n_kv_heads, G = n_q_heads / hkv;
   const int64_t n = c->len[(size_t)layer * c->p.n_seqs + seq];
   const int64_t Q = quantized_len(c, n);
-  for (int q0 = 0; q0 < n_q; q0 += NQ) {
-    const int nq = std::min(NQ, n_q - q0);
+  const int per_launch = std::max(1, std::min(NQ, MAXR / G));  // query tokens per launch
+  for (int q0 = 0; q0 < n_q; q0 += per_launch) {
+    const int nq = std::min(per_launch, n_q - q0);
     CArgs A{};
     A.seq = seq;
     A.nq = nq;

@@ -95,7 +95,8 @@ int launch_decode(const kvq_cache *c, int layer, const std::vector<DecodeSeq> &s
 size_t decode_workspace_bytes(const kvq_cache *c, int n_seqs, int n_q_heads);
 
 // Chunk attention (kvq_prefill_attn): n_q query tokens of one sequence, causal within the
-// chunk, 16 query tokens per launch; the workspace holds chunk_workspace_bytes.
+// chunk, up to 16 query tokens (80 query rows) per launch; the workspace holds
+// chunk_workspace_bytes.
 int launch_chunk(const kvq_cache *c, int layer, int seq, int n_q, int n_q_heads, const float *q, float scale,
                  float *out, void *ws, cudaStream_t st);
 size_t chunk_workspace_bytes(const kvq_cache *c, int n_q_tokens, int n_q_heads);

@@ -171,9 +171,9 @@ int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *
  * <= 0 selects 1/sqrt(128); workspace: device, >= kvq_workspace_bytes(c, n_q_tokens,
  * n_q_heads).  KVQ_E_INVAL if n_q_tokens exceeds the sequence length.  Each 32-token piece of
  * the cache is read and dequantized once (into shared memory, as f16 high part + remainder,
- * exact) for all query rows of its KV head, 16 query tokens per launch, and Q.K and P.V run as
- * dense f16 tensor-core tiles with fp32 accumulation; cached values (and the dequantized ones)
- * must lie within the f16 range (|x| < 65504). */
+ * exact) for all query rows of its KV head, up to 16 query tokens (80 query rows) per launch,
+ * and Q.K and P.V run as dense f16 tensor-core tiles with fp32 accumulation; cached values
+ * (and the dequantized ones) must lie within the f16 range (|x| < 65504). */
 int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_tokens, int32_t n_q_heads,
                      const float *q, float softmax_scale, float *out, void *workspace, size_t ws_bytes,
                      kvq_stream_t stream);
