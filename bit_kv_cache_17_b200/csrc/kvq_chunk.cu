@@ -33,10 +33,10 @@ constexpr int CH = 32;               // tokens per chunk
 constexpr int NQ = 16;               // query tokens per launch (at most MAXR / G)
 constexpr int RT = 16;               // rows per row tile (one consumer warp)
 constexpr int NC = 5;                // consumer warps: Q.K, softmax and P.V of one row tile each
-constexpr int NP = 3;                // producer warps: copies and dequantization
+constexpr int NP = 5;                // producer warps: copies and dequantization
 constexpr int MAXR = NC * RT;        // 80 rows per launch
-constexpr int NW = NP + NC;          // 8 warps
-constexpr int NT = 32 * NW;          // 256 threads
+constexpr int NW = NP + NC;          // 10 warps
+constexpr int NT = 32 * NW;          // 320 threads
 constexpr int NPT = 32 * NP;         // producer threads
 constexpr int TS = D + 8;            // padded f16 row stride of the shared tiles (272 B)
 constexpr int MAXSPL = 64;           // splits per KV head
