@@ -482,7 +482,8 @@ def run_page1_shape(args, kvq, torch, synth):
 def run_prefill(args, kvq, torch, synth):
     """Chunk attention (kvq_prefill_attn): a 64k-context kvarn4 cache (the headline data) takes
     a chunk of 16 new tokens, whose 16 queries then attend causally; timed in a CUDA graph
-    cycling layer caches.  Each 32-token piece of the cache is read once for all query rows."""
+    cycling layer caches.  Each 64-token tile of the cache is read and rebuilt once for all query
+    rows (tcgen05 tensor cores, accumulators in tensor memory)."""
     calc = LibCalc(kvq)
     cfg = synth.config2()
     n, hkv, hq, tail = cfg["n"], cfg["hkv"], cfg["hq"], cfg["tail"]

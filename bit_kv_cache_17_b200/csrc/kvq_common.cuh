@@ -123,9 +123,11 @@ struct LayerView {
 
 // Device status word bits (read and cleared by kvq_get_status): a page-table entry outside the
 // layer's page pool (the access goes to physical page 0 instead, inside the caller's buffer),
-// a merge ticket past the number of splits of its decode.
+// a merge ticket past the number of splits of its decode, a bounded wait of the chunk-attention
+// pipeline that ran out (the CTA finished without its result).
 constexpr int32_t kStatusPageTable = 1;
 constexpr int32_t kStatusTicket = 2;
+constexpr int32_t kStatusWait = 4;
 
 __device__ __forceinline__ uint8_t *subpage_ptr(const LayerView &L, int seq, int64_t page, int head,
                                                 int which) {

@@ -169,11 +169,13 @@ int kvq_decode_attn(kvq_cache *c, int32_t layer, int32_t n_seqs, const int32_t *
  * the cache as they are stored now (quantized or BF16 by the current length).
  * q: device fp32 [n_q_tokens, n_q_heads, 128]; out: device fp32, same shape; softmax_scale
  * <= 0 selects 1/sqrt(128); workspace: device, >= kvq_workspace_bytes(c, n_q_tokens,
- * n_q_heads).  KVQ_E_INVAL if n_q_tokens exceeds the sequence length.  Each 32-token piece of
- * the cache is read and dequantized once (into shared memory, as f16 high part + remainder,
- * exact) for all query rows of its KV head, up to 16 query tokens (80 query rows) per launch,
- * and Q.K and P.V run as dense f16 tensor-core tiles with fp32 accumulation; cached values
- * (and the dequantized ones) must lie within the f16 range (|x| < 65504). */
+ * n_q_heads).  KVQ_E_INVAL if n_q_tokens exceeds the sequence length.  Each 64-token tile of
+ * the cache is read and rebuilt once (into shared memory: the values with all their scales,
+ * as f16 high part + f16 remainder) for all query rows of its KV head, up to 16 query tokens
+ * (80 query rows) per launch, and Q.K and P.V run on the tcgen05 tensor cores (f16 operands,
+ * fp32 accumulators in tensor memory); cached values, the rebuilt ones and, for kvarn, the
+ * products d * t of block and token scales must lie within the f16 range (|x| < 65504).  A
+ * wait between the kernel's roles that runs out sets the status word (kvq_get_status). */
 int kvq_prefill_attn(kvq_cache *c, int32_t layer, int32_t seq, int32_t n_q_tokens, int32_t n_q_heads,
                      const float *q, float softmax_scale, float *out, void *workspace, size_t ws_bytes,
                      kvq_stream_t stream);
@@ -230,7 +232,9 @@ int kvq_locate(const kvq_cache *c, int32_t kind, int32_t layer, int32_t seq, int
  *    instead, so nothing outside dev_buf is read or written (the results of that call are
  *    wrong, the cache buffer having been corrupted);
  *  - a decode merge ticket that was not zero when the decode began (a corrupted ticket, or
- *    two decodes of one cache overlapping on the GPU): that decode's output may be stale. */
+ *    two decodes of one cache overlapping on the GPU): that decode's output may be stale;
+ *  - a wait between the roles of the chunk-attention kernel that ran out (each is bounded):
+ *    that call's output is wrong; the kernel still finishes and frees what it holds. */
 int kvq_get_status(kvq_cache *c, kvq_stream_t stream);
 
 /* Human-readable description of the cache (types, tail, bytes); valid until the next
