@@ -56,7 +56,8 @@ constexpr int PSTRIDE = 4 + D;       // floats per partial record: m, l, 2 pad, 
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float TAU = 4.f;           // lazy rescale margin (log2 units)
 constexpr uint32_t TMEM_COLS = 256;  // S buffers at columns 0 and 64, O at 128
-constexpr uint32_t WAIT_LIMIT = 1u << 22;
+constexpr uint32_t SUSPEND_NS = 100000;      // longest suspension of one mbarrier test (100 us)
+constexpr long long WAIT_CYCLES = 1ll << 31;  // a wait gives up after about a second
 
 // ---- shared memory map (bytes from a 1024-aligned base) ---------------------------------------
 // Q: rows 0..79 of q' hi at 0 and lo at QLO, core matrix (r / 8, k / 8) at (r / 8) 2048 + (k / 8) 128;
@@ -152,26 +153,29 @@ __device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
+// tests the phase; the thread is suspended (not polling) until it completes or SUSPEND_NS pass
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(SUSPEND_NS)
       : "memory");
   return ok != 0;
 }
-// Waits for the phase of the given parity to complete.  Gives up after WAIT_LIMIT polls (the
+// Waits for the phase of the given parity to complete.  Gives up after about a second (the
 // CTA's abort flag set, the status word marked); once the flag is set every wait returns at
-// once, so a CTA whose pipeline broke still runs to its end and releases its tensor memory.
+// once, so a CTA whose pipeline broke still runs to its end and releases its tensor memory
 // (follow_abort false: the wait for the tensor core's own completion, which needs no other role,
 // before the tensor memory is released)
 __device__ __forceinline__ void mbar_wait(uint32_t bar, uint32_t parity, volatile int32_t *abort, int32_t *status,
                                           bool follow_abort = true) {
-  for (uint32_t i = 0;; ++i) {
+  if (mbar_try(bar, parity)) return;
+  const long long t0 = clock64();
+  for (;;) {
     if (mbar_try(bar, parity)) return;
-    if (follow_abort && (i & 255u) == 255u && *abort) return;
-    if (i >= WAIT_LIMIT) {
+    if (follow_abort && *abort) return;
+    if (clock64() - t0 > WAIT_CYCLES) {
       *abort = 1;
       atomicOr(status, kStatusWait);
       return;
