@@ -449,47 +449,32 @@ __device__ __forceinline__ UnitIn v_load(const uint8_t *side, const RawSide &r, 
   return in;
 }
 
-// The K (V) tile of a quantized raw tile: 1024 units, four per producer thread, all four read
-// before any is computed; a warp's 32 units of one step fill four consecutive core matrices
-// (conflict-free 16-byte stores, 8 lanes per core matrix) and reads 8 tokens (quads) of the padded
-// raw rows, 8 banks apart.  K: unit u = (token 8 (u / 128) + u % 8, c8 = 4 ((u / 8) % 4) + (u / 32) % 4),
-// the lanes of a warp spanning the 4 blocks; V: (token 8 ((u / 8) % 8) + u % 8, c8 = u / 64).
+// The K (V) tile of a quantized raw tile: 1024 units, one at a time per producer thread (a
+// smaller loop body measured faster than two units in flight); a warp's 32 units fill four
+// core matrices (conflict-free 16-byte stores, 8 lanes per core matrix) and read 8 tokens
+// (quads) of the padded raw rows, 8 banks apart.  K: unit u = (token 8 (u / 128) + u % 8,
+// c8 = 4 ((u / 8) % 4) + (u / 32) % 4), the lanes of a warp spanning the 4 blocks;
+// V: (token 8 ((u / 8) % 8) + u % 8, c8 = u / 64).
 template <int FAM, int BITS>
 __device__ __forceinline__ void rebuild_k(const uint8_t *side, uint8_t *kt, int nvalid, int pt) {
   const RawSide r = raw_side(FAM, BITS, 0);
 #pragma unroll 1
-  for (int u0 = pt; u0 < 1024; u0 += 2 * NPT) {
-    UnitIn in[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int u = min(u0 + NPT * i, 1023), tok = 8 * (u >> 7) + (u & 7), c8 = 4 * ((u >> 3) & 3) + ((u >> 5) & 3);
-      in[i] = k_load<FAM, BITS>(side, r, tok, c8, tok < nvalid);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int u = u0 + NPT * i, tok = 8 * (u >> 7) + (u & 7), c8 = 4 * ((u >> 3) & 3) + ((u >> 5) & 3);
-      uint8_t *dst = kt + (tok >> 3) * 2048 + c8 * 128 + (tok & 7) * 16;
-      if (u < 1024) unit_store<FAM, BITS>(in[i], dst, dst + HALF_B);
-    }
+  for (int u = pt; u < 1024; u += NPT) {
+    const int tok = 8 * (u >> 7) + (u & 7), c8 = 4 * ((u >> 3) & 3) + ((u >> 5) & 3);
+    const UnitIn in = k_load<FAM, BITS>(side, r, tok, c8, tok < nvalid);
+    uint8_t *dst = kt + (tok >> 3) * 2048 + c8 * 128 + (tok & 7) * 16;
+    unit_store<FAM, BITS>(in, dst, dst + HALF_B);
   }
 }
 template <int FAM, int BITS>
 __device__ __forceinline__ void rebuild_v(const uint8_t *side, uint8_t *vt, int nvalid, int pt) {
   const RawSide r = raw_side(FAM, BITS, 1);
 #pragma unroll 1
-  for (int u0 = pt; u0 < 1024; u0 += 2 * NPT) {
-    UnitIn in[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int u = min(u0 + NPT * i, 1023), tok = 8 * ((u >> 3) & 7) + (u & 7), c8 = u >> 6;
-      in[i] = v_load<FAM, BITS>(side, r, tok, c8, tok < nvalid);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int u = u0 + NPT * i, tok = 8 * ((u >> 3) & 7) + (u & 7), c8 = u >> 6;
-      uint8_t *dst = vt + c8 * 1024 + (tok >> 3) * 128 + (tok & 7) * 16;
-      if (u < 1024) unit_store<FAM, BITS>(in[i], dst, dst + HALF_B);
-    }
+  for (int u = pt; u < 1024; u += NPT) {
+    const int tok = 8 * ((u >> 3) & 7) + (u & 7), c8 = u >> 6;
+    const UnitIn in = v_load<FAM, BITS>(side, r, tok, c8, tok < nvalid);
+    uint8_t *dst = vt + c8 * 1024 + (tok >> 3) * 128 + (tok & 7) * 16;
+    unit_store<FAM, BITS>(in, dst, dst + HALF_B);
   }
 }
 
