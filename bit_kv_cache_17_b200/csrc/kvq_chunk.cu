@@ -299,10 +299,6 @@ __device__ __forceinline__ void store_hilo8(uint8_t *hi, uint8_t *lo, const floa
   *reinterpret_cast<uint4 *>(lo) = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
-__device__ __forceinline__ float half_at(const uint8_t *p, int i) {
-  return __half2float(reinterpret_cast<const __half *>(p)[i]);
-}
-
 // What a unit (one token, 8 channels) reads: its code fields (one per byte, two words) and the raw
 // f16 scales: d (and t for kvarn, m for qb_1) of its (token, block), the 8 channel scales (kvarn)
 struct UnitIn {
@@ -501,6 +497,7 @@ __device__ __forceinline__ void rebuild_v_dispatch(int fam, int bits, const uint
   KVQ_EACH_QTYPE(KVQ_RV)
 #undef KVQ_RV
 }
+#undef KVQ_EACH_QTYPE
 
 // One side of a tail tile: 16-bit rows (BF16 or F16 ring) straight from global memory, four rows
 // pieces per thread loaded before any is stored; rows past the end are zero
