@@ -99,6 +99,13 @@ size_t plan(kvq_cache *c) {
   return off;
 }
 
+// the cache's metadata at creation: the identity page table and zeroed tickets / status word
+__global__ void k_init_meta(int32_t *ptab, int64_t n_ptab, uint8_t *meta, int64_t n_meta) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_ptab; i += stride) ptab[i] = (int32_t)i;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_meta; i += stride) meta[i] = 0;
+}
+
 }  // namespace
 
 namespace kvq {
@@ -207,20 +214,18 @@ int kvq_cache_create(const kvq_params *pin, void *dev_buf, size_t bytes, kvq_cac
     delete c;
     return KVQ_E_CUDA;
   }
-  // static page table: sequence s, logical page j -> physical page s * max_pages + j
-  if (c->max_pages > 0) {
-    std::vector<int32_t> ptab((size_t)p->n_seqs * c->max_pages);
-    for (size_t i = 0; i < ptab.size(); ++i) ptab[i] = (int32_t)i;
-    if (cudaMemcpy(c->base + c->off_ptab, ptab.data(), ptab.size() * sizeof(int32_t),
-                   cudaMemcpyHostToDevice) != cudaSuccess) {
-      delete c;
-      return KVQ_E_CUDA;
-    }
-  }
-  if (cudaMemset(c->base + c->off_tickets, 0, c->total - c->off_tickets) != cudaSuccess) {
+  // the metadata, by one kernel on the legacy default stream (no host copy, no wait): the
+  // static page table (sequence s, logical page j -> physical page s * max_pages + j), the
+  // merge tickets and the status word at zero
+  const int64_t n_ptab = (int64_t)p->n_seqs * c->max_pages;
+  const int64_t n_meta = (int64_t)(c->total - c->off_tickets);
+  k_init_meta<<<(unsigned)std::max<int64_t>(1, std::min<int64_t>(4 * c->num_sms, (std::max(n_ptab, n_meta) + 255) / 256)),
+                256>>>(reinterpret_cast<int32_t *>(c->base + c->off_ptab), n_ptab, c->base + c->off_tickets, n_meta);
+  if (cudaGetLastError() != cudaSuccess) {
     delete c;
     return KVQ_E_CUDA;
   }
+  kvq::note_launches(1);
   *out = c;
   return KVQ_OK;
 }

@@ -125,8 +125,10 @@ int kvq_payload_bytes(int32_t type, int32_t raw_bits, int64_t n_layers, int64_t 
                       int64_t n, int64_t tail, double *bytes);
 
 /* Creates a cache inside the caller's device buffer dev_buf (bytes >= kvq_cache_bytes).
- * Zero-fills the metadata part of dev_buf (synchronous on the current device).  All
- * sequences start empty.  *out receives a host handle. */
+ * The metadata part of dev_buf (page table, merge tickets, status word) is initialized by
+ * one kernel enqueued on the current device's legacy default stream (no host copy, no wait):
+ * work on streams that do not synchronize with it (cudaStreamNonBlocking) must be ordered
+ * after it by the caller.  All sequences start empty.  *out receives a host handle. */
 int kvq_cache_create(const kvq_params *p, void *dev_buf, size_t bytes, kvq_cache **out);
 
 /* Frees the host handle only; dev_buf stays owned by the caller. */
